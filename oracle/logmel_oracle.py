@@ -138,9 +138,12 @@ def power_spectrum(frames_windowed: np.ndarray) -> np.ndarray:
 
 # --- step 4: filterbank -----------------------------------------------------
 def mel_edges(p: Params = DEFAULT) -> np.ndarray:
-    """n_mels + 2 edge frequencies (Hz), uniform on the mel scale over fmin..fmax."""
+    """n_mels + 2 edge frequencies (Hz), uniform on the mel scale over fmin..fmax;
+    the end edges are fmin and fmax themselves (not their mel round trip)."""
     m = np.linspace(hz_to_mel(p.fmin), hz_to_mel(p.fmax), p.n_mels + 2)
-    return mel_to_hz(m)
+    e = mel_to_hz(m)
+    e[0], e[-1] = p.fmin, p.fmax
+    return e
 
 
 def mel_filterbank(p: Params = DEFAULT) -> np.ndarray:
