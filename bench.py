@@ -1,0 +1,314 @@
+"""Throughput of the batched log-mel spectrogram on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one pass of the whole path (framing, window, FFT, power, mel, log)
+over one batch: 64 speech-like clips of 30 s (480000 fp32 samples each,
+191,872 frames) per GPU, inputs resident in HBM, L2 flushed between steps.
+Prints one JSON line (rank 0).  For N > 1 launch with torchrun; each rank
+processes its own batch (weak scaling, no collective on the data path).
+
+``--impl reference`` times the float64 CPU oracle on the host cores on a
+bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "log-mel frames/sec and audio-sec/sec on 1 B200; % of HBM/FP32 roofline"
+UNIT = "frames/s"
+N_CLIPS, CLIP = 64, W.CLIP_30S
+FRAMES_PER_CLIP = (CLIP - 400) // 160 + 1            # 2998
+N_MELS = 128
+WORKLOAD = "dense batch: 64 speech-like clips x 30 s (480000 fp32 samples each) per GPU"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def algorithmic_bytes(n_samples: int, n_frames: int, n_utt: int) -> int:
+    """Each input sample read once, each output value written once, plus the
+    per-utterance metadata (sample, frame and tile offsets)."""
+    return 4 * n_samples + 4 * N_MELS * n_frames + 20 * (n_utt + 1)
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in ("log_mel_spectrogram_logmel_b200/csrc/logmel_kernel.cuh",
+                "log_mel_spectrogram_logmel_b200/csrc/logmel.cu"):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic():
+    """DRAM bytes per launch of the fused kernel from the committed ncu summary,
+    if it was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return d.get("dram_bytes_per_launch_full_step")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML while running."""
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._period = period_s
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception as e:  # noqa: BLE001
+            self.error = repr(e)
+
+    def _run(self):
+        nv = self._nv
+        names = {
+            "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+            "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+            "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        }
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for k, bit in names.items():
+                    if r & bit and k != "gpu_idle":
+                        self.reasons.add(k)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self._ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def cpu_oracle_rate(budget_s: float, frames_cap: int):
+    """The float64 oracle, as it stands, on clips of the same workload: frames/s."""
+    import oracle as O
+    cores = len(os.sched_getaffinity(0))
+    frames, t0, i = 0, time.perf_counter(), 0
+    clip = W.speech_like(CLIP, 1000)
+    n = min(frames_cap, FRAMES_PER_CLIP)
+    sub = clip[:160 * (n - 1) + 400]
+    O.log_mel(sub[:4000])                       # warm the cached tables
+    t0 = time.perf_counter()
+    while True:
+        O.log_mel(sub)
+        frames += n
+        i += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return frames / dt, cores, f"{i} passes of the oracle over a {n}-frame prefix of one 30 s clip ({frames} frames, {dt:.1f} s)"
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    budget = 90.0
+    per_step_frames = int(max(98, min(FRAMES_PER_CLIP, budget / max(1, args.steps + args.warmup) / 1e-5)))
+    import oracle as O
+    clip = W.speech_like(CLIP, 1000)
+    sub = clip[:160 * (per_step_frames - 1) + 400]
+    for _ in range(args.warmup):
+        O.log_mel(sub)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        O.log_mel(sub)
+    dt = time.perf_counter() - t0
+    value = per_step_frames * args.steps / dt
+    cores = len(os.sched_getaffinity(0))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "audio_s_per_s": value * 160 / 16000,
+        "config": {"workload": WORKLOAD, "sample": f"{per_step_frames} frames of one clip per step"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{per_step_frames}-frame prefix of one 30 s clip per step, {args.steps} steps"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=30)
+    ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+
+    import torch
+    import log_mel_spectrogram_logmel_b200 as lm
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+
+    pcm_h, off = W.dense_batch(N_CLIPS, CLIP, seed0=1000 + 100_000 * rank)
+    n_samples = pcm_h.size
+    frames = N_CLIPS * FRAMES_PER_CLIP
+    pcm = torch.from_numpy(pcm_h).to(dev)
+    plan = lm.Plan(device=dev)
+    out = torch.empty((frames, N_MELS), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(args.warmup):
+        plan.compute(pcm, off, out=out)
+    torch.cuda.synchronize(dev)
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    with sampler:
+        for i in range(args.steps):
+            flush.fill_(float(i))                       # evict L2 between steps (not timed)
+            starts[i].record(stream)
+            plan.compute(pcm, off, out=out)
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+    if pg:
+        pg.barrier()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = float(sum(step_ms))
+    if pg:
+        t = torch.tensor([total_ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = frames * world * args.steps / (total_ms / 1e3)
+
+    # ---- e2e: host buffers through the public API, copies inside the timed region
+    pcm_pin = torch.from_numpy(pcm_h).pin_memory()
+    out_pin = torch.empty((frames, N_MELS), dtype=torch.float32).pin_memory()
+    pcm_dev = torch.empty_like(pcm)
+    for _ in range(3):
+        pcm_dev.copy_(pcm_pin, non_blocking=True)
+        plan.compute(pcm_dev, off, out=out)
+        out_pin.copy_(out, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    if pg:
+        pg.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        pcm_dev.copy_(pcm_pin, non_blocking=True)
+        plan.compute(pcm_dev, off, out=out)
+        out_pin.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    if pg:
+        t = torch.tensor([e2e_ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = frames * world * args.e2e_steps / (e2e_ms / 1e3)
+
+    if rank == 0:
+        peaks, peak_kind = measured_peaks()
+        bytes_launch = algorithmic_bytes(n_samples, frames, N_CLIPS)
+        achieved = bytes_launch / (ms_per_step / 1e3) / 1e9
+        peak = float(peaks["hbm_gbs"])
+        cpu_value, cores, sample = cpu_oracle_rate(args.cpu_budget_s, FRAMES_PER_CLIP) if world == 1 else (None, None, None)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "audio_s_per_s": value * 160 / 16000,
+            "config": {"workload": WORKLOAD, "n_utt": N_CLIPS, "frames_per_step_per_gpu": frames,
+                       "samples_per_step_per_gpu": n_samples, "n_mels": N_MELS,
+                       "l2": "flushed between steps (256 MiB write, untimed)",
+                       "parallelism": f"dp{world} (independent batches, no collective)"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": ncu_traffic(),
+                         "peak_source": f"{peak_kind} hbm_gbs (burst copy)",
+                         "algorithmic_bytes_per_launch": bytes_launch,
+                         "kernel": "logmel_fused_kernel (1 launch per step; event pair brackets the "
+                                   "call's metadata copy and the kernel)"},
+            "cpu_baseline": ({"value": cpu_value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                              "sample": sample} if cpu_value else None),
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": 4 * n_samples,
+                    "d2h_bytes_per_step": 4 * N_MELS * frames, "steps": args.e2e_steps},
+            "gpu_launches": args.steps,
+            "clocks": sampler.summary(),
+            "step_ms_min": min(step_ms), "step_ms_median": statistics.median(step_ms),
+        }
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

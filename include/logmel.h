@@ -1,0 +1,162 @@
+/*
+ * logmel.h -- C ABI of the B200 (sm_100a) batched log-mel spectrogram.
+ *
+ * The operation is the log-mel front-end that "从零理解 ASR：音频基础、
+ * Qwen3-ASR 架构，以及离线 vs 流式推理原理" defines in section 2.3
+ * ("Log-Mel Spectrogram 提取流水线", steps 1-5):
+ *   16 kHz mono fp32 PCM -> frames of n_fft = 400 samples every hop = 160
+ *   samples, no padding, floor((N - 400) / 160) + 1 frames (step 1)
+ *   -> symmetric Hamming window 0.54 - 0.46 cos(2 pi n / 399) (step 2)
+ *   -> real DFT to 201 bins, power |X|^2 (step 3)
+ *   -> 128 triangular filters uniform on mel = 2595 log10(1 + f / 700)
+ *      over fmin..fmax, linear in Hz, unnormalised (step 4)
+ *   -> ln(max(mel_energy, 1e-10)) (step 5)
+ * Output is fp32, frames-major [frames, n_mels] (the section's shape flow
+ * [3000, 400] -> [3000, 201] -> [3000, 128]).
+ *
+ * Streaming follows the chunked input of section 6 of the same page and
+ * the 80 / 120 / 160 ms audio clocks of the "Audio8-ASR-Infinite" page:
+ * after each push the stream emits every frame that the audio received so
+ * far completes, and carries the unconsumed samples (240..399 of them once
+ * 400 samples have arrived) to the next push.  Streaming output equals the
+ * offline output on the concatenated audio bit for bit.
+ *
+ * Conventions (all entry points):
+ *   - Every pointer documented "device" must be memory of the plan's device;
+ *     "host" pointers are ordinary host memory.  All work is enqueued on the
+ *     caller's `stream` (a cudaStream_t, passed as void*; NULL = the legacy
+ *     default stream); no entry point synchronises the device unless its
+ *     comment says so.
+ *   - The caller owns every input and output buffer.  A plan owns its
+ *     constant tables and scratch; a logmel_stream owns its carry state.
+ *   - A plan or stream object must not be used from two host threads at the
+ *     same time.  Calls on one object must be ordered on the GPU (one CUDA
+ *     stream, or explicit synchronisation between streams).
+ *   - Errors are returned as logmel_status; nothing is truncated silently:
+ *     sizes the kernels cannot index return LOGMEL_ERR_INPUT_TOO_LONG.
+ *     On an error return nothing has been enqueued.
+ */
+#ifndef LOGMEL_H_
+#define LOGMEL_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LOGMEL_OK = 0,
+  LOGMEL_ERR_INVALID_ARG = 1,    /* null pointer, bad offsets, bad size      */
+  LOGMEL_ERR_UNSUPPORTED = 2,    /* parameters outside what the kernels do   */
+  LOGMEL_ERR_CUDA = 3,           /* a CUDA runtime call failed               */
+  LOGMEL_ERR_OOM = 4,            /* device or pinned allocation failed       */
+  LOGMEL_ERR_INPUT_TOO_LONG = 5, /* a count exceeds the kernels' index range */
+  LOGMEL_ERR_DEVICE_STATUS = 6   /* a kernel flagged an inconsistency        */
+} logmel_status;
+
+typedef struct logmel_plan logmel_plan;
+typedef struct logmel_stream logmel_stream;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* logmel_status_string(logmel_status s);
+
+/* Creates a plan on the current CUDA device: builds the Hamming window,
+ * FFT twiddles and the mel filterbank in float64 on the host, rounds them
+ * to fp32 and uploads them (section 2.3, steps 2-4; preprocessor config
+ * n_mels 128, n_fft 400, hop 160).
+ *   sr      sample rate in Hz (> 0); it places bin k at k * sr / n_fft Hz
+ *   n_fft   must be 400          (else LOGMEL_ERR_UNSUPPORTED)
+ *   hop     must be 160          (else LOGMEL_ERR_UNSUPPORTED)
+ *   n_mels  1..201               (else LOGMEL_ERR_UNSUPPORTED)
+ *   fmin, fmax  0 <= fmin < fmax <= sr / 2 (else LOGMEL_ERR_INVALID_ARG)
+ * On success *out owns device memory until logmel_plan_destroy. */
+logmel_status logmel_plan_create(int sr, int n_fft, int hop, int n_mels, float fmin, float fmax,
+                                 logmel_plan** out);
+
+/* Frees the plan (synchronises the plan's device first).  NULL is a no-op. */
+void logmel_plan_destroy(logmel_plan* plan);
+
+/* floor((n_samples - n_fft) / hop) + 1, or 0 if n_samples < n_fft
+ * (section 2.3 step 1; no padding).  Returns -1 for a NULL plan. */
+int64_t logmel_num_frames(const logmel_plan* plan, int64_t n_samples);
+
+/* Frame offsets of a ragged batch: offsets (host, n_utt + 1 entries, CSR,
+ * non-decreasing, offsets[0] may be non-zero) -> frame_offsets (host,
+ * n_utt + 1 entries, frame_offsets[0] = 0, exclusive prefix sum of the
+ * per-utterance frame counts).  Pure host function. */
+logmel_status logmel_frame_offsets(const logmel_plan* plan, const int64_t* offsets, int64_t n_utt,
+                                   int64_t* frame_offsets);
+
+/* Offline ragged batch.  Utterance u is pcm[offsets[u] .. offsets[u+1]).
+ *   pcm      device, fp32, at least offsets[n_utt] samples
+ *   offsets  host, int64, n_utt + 1 entries, non-decreasing, offsets[0] >= 0
+ *   out      device, fp32 [total_frames, n_mels] row-major, where
+ *            total_frames = sum of logmel_num_frames over utterances; the
+ *            rows of utterance u start at frame_offsets[u]
+ * Utterances shorter than n_fft contribute no rows and no error.  The call
+ * copies a few bytes of tile metadata host->device on `stream` (from a
+ * pinned ring owned by the plan) and launches one kernel; it does not
+ * synchronise unless the plan's scratch must grow (first call with a larger
+ * batch), which synchronises the device.  n_utt == 0 or total_frames == 0
+ * is a no-op. */
+logmel_status logmel_compute(logmel_plan* plan, const float* pcm, const int64_t* offsets,
+                             int64_t n_utt, float* out, void* stream);
+
+/* Total output rows logmel_compute writes for these offsets (host). */
+int64_t logmel_total_frames(const logmel_plan* plan, const int64_t* offsets, int64_t n_utt);
+
+/* Streaming state for n_streams independent streams (device carry of up to
+ * n_fft - 1 samples per stream; zero-initialised: every stream is empty). */
+logmel_status logmel_stream_create(logmel_plan* plan, int n_streams, logmel_stream** out);
+void logmel_stream_destroy(logmel_stream* st);
+
+/* Frames the next push of `len` samples to stream `stream_id` will emit
+ * (host bookkeeping only; -1 on a bad argument). */
+int64_t logmel_stream_frames_for_push(const logmel_stream* st, int stream_id, int64_t len);
+
+/* Pushes `len` samples (device, fp32) to one stream.  Emits n frames into
+ * out (device, fp32 [out_capacity, n_mels]); *n_frames_out (host) receives
+ * n, computed on the host, so no synchronisation is needed.  Returns
+ * LOGMEL_ERR_INVALID_ARG if n > out_capacity (nothing enqueued). */
+logmel_status logmel_stream_push(logmel_stream* st, int stream_id, const float* chunk, int64_t len,
+                                 float* out, int64_t out_capacity, int64_t* n_frames_out,
+                                 void* stream);
+
+/* Pushes one chunk to every stream at once.
+ *   chunks         device, fp32 [n_streams, chunk_stride], row s = stream s,
+ *                  the first `len` samples of each row are pushed
+ *   out            device, fp32 [n_streams, out_capacity, n_mels]; stream s
+ *                  writes its n_frames_out[s] rows at out + s*out_capacity*n_mels
+ *   n_frames_out   host, int64 [n_streams], filled before the call returns
+ * All streams advance by `len` samples.  Returns LOGMEL_ERR_INVALID_ARG if
+ * any stream would emit more than out_capacity frames. */
+logmel_status logmel_stream_push_batch(logmel_stream* st, const float* chunks, int64_t chunk_stride,
+                                       int64_t len, float* out, int64_t out_capacity,
+                                       int64_t* n_frames_out, void* stream);
+
+/* Largest per-stream frame count the next push_batch of `len` samples emits. */
+int64_t logmel_stream_max_frames(const logmel_stream* st, int64_t len);
+
+/* Checkpoint / resume of the carry state.  logmel_stream_state_bytes gives
+ * the size of the opaque blob; get_state synchronises `stream` and copies
+ * the state into host memory; set_state uploads a blob written by
+ * get_state for the same n_streams (else LOGMEL_ERR_INVALID_ARG).  A
+ * resumed stream produces output bit-identical to an uninterrupted one. */
+int64_t logmel_stream_state_bytes(const logmel_stream* st);
+logmel_status logmel_stream_get_state(logmel_stream* st, void* host_blob, int64_t bytes, void* stream);
+logmel_status logmel_stream_set_state(logmel_stream* st, const void* host_blob, int64_t bytes,
+                                      void* stream);
+
+/* Empties one stream (or all streams if stream_id < 0), enqueued on `stream`. */
+logmel_status logmel_stream_reset(logmel_stream* st, int stream_id, void* stream);
+
+/* Reads and clears the plan's device status word (synchronises `stream`).
+ * *code = 0 when no kernel has flagged an inconsistency since the last read. */
+logmel_status logmel_plan_device_status(logmel_plan* plan, int* code, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LOGMEL_H_ */

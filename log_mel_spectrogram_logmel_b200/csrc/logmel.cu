@@ -1,0 +1,667 @@
+// C ABI of the batched log-mel spectrogram (declared in include/logmel.h).
+//
+// Host side: plan creation (window, FFT twiddles and the mel filterbank of
+// "从零理解 ASR：音频基础、Qwen3-ASR 架构，以及离线 vs 流式推理原理" section 2.3,
+// built in float64 and rounded to fp32), the ragged-batch index map (frame
+// and tile prefix sums), the streaming carry state and its checkpoint blob.
+// Device side: logmel_kernel.cuh.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "logmel.h"
+#include "logmel_kernel.cuh"
+
+using namespace logmel;
+
+namespace {
+
+constexpr int RING = 4;
+constexpr uint32_t STATE_MAGIC = 0x314d4c53u;   // "SLM1"
+
+struct PinnedSlot {
+  unsigned char* host = nullptr;
+  cudaEvent_t done = nullptr;
+  bool used = false;
+};
+
+struct MetaView {
+  int64_t* sample_off;
+  int64_t* frame_off;
+  int* tile_off;
+};
+
+size_t meta_bytes(int64_t n_utt) {
+  const size_t n = (size_t)n_utt + 1;
+  size_t b = 16 * n;                 // two int64 arrays
+  b += (4 * n + 15) & ~size_t(15);   // int32 tile offsets
+  return b;
+}
+
+MetaView meta_view(unsigned char* base, int64_t n_utt) {
+  const size_t n = (size_t)n_utt + 1;
+  MetaView v;
+  v.sample_off = reinterpret_cast<int64_t*>(base);
+  v.frame_off = reinterpret_cast<int64_t*>(base + 8 * n);
+  v.tile_off = reinterpret_cast<int*>(base + 16 * n);
+  return v;
+}
+
+// cos and sin of 2 pi num / den, exact at multiples of pi / 2.
+void cos_sin_2pi(long num, long den, double* c, double* s) {
+  num %= den;
+  if (num < 0) num += den;
+  if (4 * num % den == 0) {
+    const int q = (int)(4 * num / den);
+    const double cs[4] = {1, 0, -1, 0}, sn[4] = {0, 1, 0, -1};
+    *c = cs[q];
+    *s = sn[q];
+    return;
+  }
+  const double a = 2.0 * M_PI * (double)num / (double)den;
+  *c = std::cos(a);
+  *s = std::sin(a);
+}
+
+double hz_to_mel(double f) { return 2595.0 * std::log10(1.0 + f / 700.0); }
+double mel_to_hz(double m) { return 700.0 * (std::pow(10.0, m / 2595.0) - 1.0); }
+
+int64_t frames_of(int64_t n) { return n < NFFT ? 0 : (n - NFFT) / HOP + 1; }
+
+}  // namespace
+
+struct logmel_plan {
+  int sr = 0, n_fft = 0, hop = 0, n_mels = 0;
+  float fmin = 0.f, fmax = 0.f;
+  int device = 0;
+  int max_ctas = 0;
+  size_t smem_bytes = 0;
+  Tables* d_tables = nullptr;
+  int* d_status = nullptr;
+  unsigned char* d_meta = nullptr;
+  size_t meta_cap = 0;
+  PinnedSlot ring[RING];
+  size_t ring_cap = 0;
+  int ring_next = 0;
+  Args mel{};               // filterbank fields copied into every launch
+  bool default_mel = false; // structure equals the compiled default layout
+};
+
+struct logmel_stream {
+  logmel_plan* plan = nullptr;
+  int n_streams = 0;
+  float* d_carry = nullptr;
+  int* d_carry_len = nullptr;
+  std::vector<int64_t> total;    // samples received per stream
+  std::vector<int> carry_len;    // host mirror of d_carry_len
+};
+
+// ---------------------------------------------------------------------------
+// small kernels
+// ---------------------------------------------------------------------------
+namespace {
+
+// New carry after a push whose frames were computed with the carry left in
+// place (pushes emitting more than one tile per stream): one CTA per stream.
+__global__ void carry_update_kernel(float* carry, int* carry_len, const float* chunks,
+                                    int64_t chunk_stride, int64_t len, int stream_base) {
+  __shared__ float buf[CARRY_CAP];
+  const int sl = blockIdx.x;
+  const int s = stream_base + sl;
+  float* cs = carry + (int64_t)s * CARRY_CAP;
+  const float* ch = chunks + (int64_t)sl * chunk_stride;
+  const int c = carry_len[s];            // read by every thread before the barrier
+  const int64_t B = c + len;
+  const int64_t nf = B >= NFFT ? (B - NFFT) / HOP + 1 : 0;
+  const int L = (int)(B - nf * HOP);     // < 400
+  const int64_t from = nf * HOP;
+  for (int i = threadIdx.x; i < L; i += blockDim.x) {
+    const int64_t q = from + i;
+    buf[i] = q < c ? cs[q] : ch[q - c];
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < L; i += blockDim.x) cs[i] = buf[i];
+  if (threadIdx.x == 0) carry_len[s] = L;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// C ABI
+// ---------------------------------------------------------------------------
+#define CK(call)                                   \
+  do {                                             \
+    cudaError_t e_ = (call);                       \
+    if (e_ != cudaSuccess) return LOGMEL_ERR_CUDA; \
+  } while (0)
+
+extern "C" {
+
+const char* logmel_status_string(logmel_status s) {
+  switch (s) {
+    case LOGMEL_OK: return "ok";
+    case LOGMEL_ERR_INVALID_ARG: return "invalid argument";
+    case LOGMEL_ERR_UNSUPPORTED: return "unsupported parameters";
+    case LOGMEL_ERR_CUDA: return "CUDA runtime error";
+    case LOGMEL_ERR_OOM: return "out of memory";
+    case LOGMEL_ERR_INPUT_TOO_LONG: return "input too long for the kernels' index range";
+    case LOGMEL_ERR_DEVICE_STATUS: return "a kernel flagged an inconsistency";
+  }
+  return "unknown status";
+}
+
+static logmel_status build_tables(Tables* t) {
+  std::memset(t, 0, sizeof(Tables));
+  // window pairs for pass A: sample n = 20 m1 + 2 m2 and n + 1
+  for (int m2 = 0; m2 < N2; ++m2)
+    for (int m1 = 0; m1 < N1; ++m1) {
+      const int n = 2 * (N2 * m1 + m2);
+      const double w0 = 0.54 - 0.46 * std::cos(2.0 * M_PI * n / (NFFT - 1));
+      const double w1 = 0.54 - 0.46 * std::cos(2.0 * M_PI * (n + 1) / (NFFT - 1));
+      t->win[m2][m1] = make_float2((float)w0, (float)w1);
+    }
+  // pass-A twiddles e^{-2 pi i m2 k1 / 200} = c - i s
+  for (int m2 = 0; m2 < N2; ++m2)
+    for (int k1 = 0; k1 < N1; ++k1) {
+      double c, s;
+      cos_sin_2pi((long)m2 * k1, NFFT / 2, &c, &s);
+      t->tw[m2][k1] = make_float4((float)c, (float)c, (float)s, (float)s);
+      t->twn[m2][k1] = make_float2((float)-s, (float)-s);
+    }
+  // real-split twiddles u_k = -i e^{-2 pi i k / 400} = -sin - i cos
+  for (int k = 0; k < NFFT / 2; ++k) {
+    double c, s;
+    cos_sin_2pi(k, NFFT, &c, &s);
+    const double ur = -s, ui = -c;
+    t->post[k] = make_float4((float)ur, (float)ur, (float)ui, (float)ui);
+    t->postn[k] = make_float2((float)-ui, (float)-ui);
+  }
+  return LOGMEL_OK;
+}
+
+}  // extern "C"
+
+// Triangular filters, linear in Hz between mel-spaced edges, unnormalised
+// (section 2.3 step 4), stored as contiguous nonzero runs per band; weights
+// carry the factor 1/4 of the real split (which yields |2 X|^2).  Also the
+// split of the bands over the mel warps (cost per band = nonzeros + 3).
+static logmel_status build_mel(logmel_plan* p) {
+  Args& a = p->mel;
+  const int nm = p->n_mels;
+  std::vector<double> edge(nm + 2);
+  const double m_lo = hz_to_mel(p->fmin), m_hi = hz_to_mel(p->fmax);
+  for (int j = 0; j < nm + 2; ++j) edge[j] = mel_to_hz(m_lo + (m_hi - m_lo) * j / (nm + 1));
+  edge[0] = p->fmin;          // the end edges are fmin and fmax exactly
+  edge[nm + 1] = p->fmax;
+  int woff = 0;
+  std::vector<int> cost(nm);
+  for (int m = 0; m < nm; ++m) {
+    int lo = -1, cnt = 0;
+    for (int k = 0; k < NBINS; ++k) {
+      const double f = (double)k * p->sr / NFFT;
+      const double rise = (f - edge[m]) / (edge[m + 1] - edge[m]);
+      const double fall = (edge[m + 2] - f) / (edge[m + 2] - edge[m + 1]);
+      const double h = std::max(0.0, std::min(rise, fall));
+      if (h > 0.0) {
+        if (k == 0 || k == NBINS - 1) return LOGMEL_ERR_UNSUPPORTED;   // edge bins never weigh
+        if (lo < 0) lo = k;
+        if (k != lo + cnt) return LOGMEL_ERR_UNSUPPORTED;              // not contiguous
+        if (woff + cnt >= MAX_WEIGHTS) return LOGMEL_ERR_UNSUPPORTED;
+        a.mel_w[woff + cnt] = (float)h * 0.25f;
+        ++cnt;
+      }
+    }
+    a.mel_lo[m] = (short)(lo < 0 ? 1 : lo);
+    a.mel_cnt[m] = (short)cnt;
+    a.mel_woff[m] = (short)woff;
+    woff += cnt;
+    cost[m] = cnt + 3;
+  }
+  long total = 0;
+  for (int m = 0; m < nm; ++m) total += cost[m];
+  a.warp_band[0] = 0;
+  long run = 0;
+  int m = 0;
+  for (int w = 1; w < MEL_WARPS; ++w) {
+    const long target = total * w / MEL_WARPS;
+    while (m < nm && run + cost[m] / 2 < target) run += cost[m++];
+    a.warp_band[w] = (short)m;
+  }
+  a.warp_band[MEL_WARPS] = (short)nm;
+  // the unrolled path applies when the structure equals the compiled one
+  bool same = nm == mel_default::N_MELS && woff == mel_default::NNZ;
+  for (int i = 0; same && i < nm; ++i)
+    same = (mel_default::CNT[i] == a.mel_cnt[i]) && (mel_default::WOFF[i] == a.mel_woff[i]) &&
+           (mel_default::CNT[i] == 0 || mel_default::LO[i] == a.mel_lo[i]);
+  for (int w = 0; same && w <= MEL_WARPS; ++w) same = mel_default::WARP_BAND[w] == a.warp_band[w];
+  p->default_mel = same;
+  return LOGMEL_OK;
+}
+
+template <bool kDefault>
+static logmel_status setup_kernel(logmel_plan* p, int sms) {
+  if (cudaFuncSetAttribute(logmel_fused_kernel<kDefault>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)p->smem_bytes) != cudaSuccess)
+    return LOGMEL_ERR_CUDA;
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, logmel_fused_kernel<kDefault>, THREADS,
+                                                    p->smem_bytes) != cudaSuccess ||
+      occ < 1)
+    return LOGMEL_ERR_CUDA;
+  p->max_ctas = sms * occ;
+  return LOGMEL_OK;
+}
+
+static cudaError_t launch(const logmel_plan* p, Args& a, int grid, cudaStream_t s) {
+  std::memcpy(a.mel_w, p->mel.mel_w, sizeof a.mel_w);
+  std::memcpy(a.mel_lo, p->mel.mel_lo, sizeof a.mel_lo);
+  std::memcpy(a.mel_cnt, p->mel.mel_cnt, sizeof a.mel_cnt);
+  std::memcpy(a.mel_woff, p->mel.mel_woff, sizeof a.mel_woff);
+  std::memcpy(a.warp_band, p->mel.warp_band, sizeof a.warp_band);
+  if (p->default_mel)
+    logmel_fused_kernel<true><<<grid, THREADS, p->smem_bytes, s>>>(a);
+  else
+    logmel_fused_kernel<false><<<grid, THREADS, p->smem_bytes, s>>>(a);
+  return cudaGetLastError();
+}
+
+extern "C" {
+
+logmel_status logmel_plan_create(int sr, int n_fft, int hop, int n_mels, float fmin, float fmax,
+                                 logmel_plan** out) {
+  if (!out) return LOGMEL_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (sr <= 0 || !(fmin >= 0.f) || !(fmax > fmin) || (double)fmax > sr / 2.0)
+    return LOGMEL_ERR_INVALID_ARG;
+  if (n_fft != NFFT || hop != HOP || n_mels < 1 || n_mels > MAX_MELS) return LOGMEL_ERR_UNSUPPORTED;
+  logmel_plan* p = new (std::nothrow) logmel_plan();
+  if (!p) return LOGMEL_ERR_OOM;
+  p->sr = sr;
+  p->n_fft = n_fft;
+  p->hop = hop;
+  p->n_mels = n_mels;
+  p->fmin = fmin;
+  p->fmax = fmax;
+  Tables* t = new (std::nothrow) Tables();
+  if (!t) {
+    delete p;
+    return LOGMEL_ERR_OOM;
+  }
+  logmel_status st = build_tables(t);
+  if (st == LOGMEL_OK) st = build_mel(p);
+  if (st != LOGMEL_OK) {
+    delete t;
+    delete p;
+    return st;
+  }
+  auto fail = [&](logmel_status s) {
+    delete t;
+    logmel_plan_destroy(p);
+    return s;
+  };
+  if (cudaGetDevice(&p->device) != cudaSuccess) return fail(LOGMEL_ERR_CUDA);
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, p->device) != cudaSuccess)
+    return fail(LOGMEL_ERR_CUDA);
+  p->smem_bytes = sizeof(Smem);
+  st = p->default_mel ? setup_kernel<true>(p, sms) : setup_kernel<false>(p, sms);
+  if (st != LOGMEL_OK) return fail(st);
+  if (cudaMalloc(&p->d_tables, sizeof(Tables)) != cudaSuccess) return fail(LOGMEL_ERR_OOM);
+  if (cudaMalloc(&p->d_status, sizeof(int)) != cudaSuccess) return fail(LOGMEL_ERR_OOM);
+  if (cudaMemcpy(p->d_tables, t, sizeof(Tables), cudaMemcpyHostToDevice) != cudaSuccess)
+    return fail(LOGMEL_ERR_CUDA);
+  if (cudaMemset(p->d_status, 0, sizeof(int)) != cudaSuccess) return fail(LOGMEL_ERR_CUDA);
+  for (int i = 0; i < RING; ++i)
+    if (cudaEventCreateWithFlags(&p->ring[i].done, cudaEventDisableTiming) != cudaSuccess)
+      return fail(LOGMEL_ERR_CUDA);
+  delete t;
+  *out = p;
+  return LOGMEL_OK;
+}
+
+void logmel_plan_destroy(logmel_plan* p) {
+  if (!p) return;
+  int prev = -1;
+  cudaGetDevice(&prev);
+  cudaSetDevice(p->device);
+  cudaDeviceSynchronize();
+  cudaFree(p->d_tables);
+  cudaFree(p->d_status);
+  cudaFree(p->d_meta);
+  for (int i = 0; i < RING; ++i) {
+    if (p->ring[i].host) cudaFreeHost(p->ring[i].host);
+    if (p->ring[i].done) cudaEventDestroy(p->ring[i].done);
+  }
+  if (prev >= 0) cudaSetDevice(prev);
+  delete p;
+}
+
+int64_t logmel_num_frames(const logmel_plan* p, int64_t n) {
+  if (!p) return -1;
+  return n < 0 ? 0 : frames_of(n);
+}
+
+static logmel_status check_offsets(const int64_t* off, int64_t n_utt) {
+  if (!off || n_utt < 0) return LOGMEL_ERR_INVALID_ARG;
+  if (n_utt == 0) return LOGMEL_OK;
+  if (off[0] < 0) return LOGMEL_ERR_INVALID_ARG;
+  for (int64_t u = 0; u < n_utt; ++u)
+    if (off[u + 1] < off[u]) return LOGMEL_ERR_INVALID_ARG;
+  return LOGMEL_OK;
+}
+
+logmel_status logmel_frame_offsets(const logmel_plan* p, const int64_t* off, int64_t n_utt,
+                                   int64_t* fo) {
+  if (!p || !fo) return LOGMEL_ERR_INVALID_ARG;
+  logmel_status st = check_offsets(off, n_utt);
+  if (st != LOGMEL_OK) return st;
+  fo[0] = 0;
+  for (int64_t u = 0; u < n_utt; ++u) fo[u + 1] = fo[u] + frames_of(off[u + 1] - off[u]);
+  return LOGMEL_OK;
+}
+
+int64_t logmel_total_frames(const logmel_plan* p, const int64_t* off, int64_t n_utt) {
+  if (!p || check_offsets(off, n_utt) != LOGMEL_OK) return -1;
+  int64_t t = 0;
+  for (int64_t u = 0; u < n_utt; ++u) t += frames_of(off[u + 1] - off[u]);
+  return t;
+}
+
+static logmel_status ensure_meta(logmel_plan* p, size_t bytes) {
+  if (bytes > p->ring_cap) {
+    for (int i = 0; i < RING; ++i) {
+      if (p->ring[i].used) CK(cudaEventSynchronize(p->ring[i].done));
+      if (p->ring[i].host) cudaFreeHost(p->ring[i].host);
+      p->ring[i].host = nullptr;
+      p->ring[i].used = false;
+    }
+    size_t cap = std::max<size_t>(bytes, 4096);
+    for (int i = 0; i < RING; ++i)
+      if (cudaHostAlloc(&p->ring[i].host, cap, cudaHostAllocDefault) != cudaSuccess) {
+        p->ring_cap = 0;
+        return LOGMEL_ERR_OOM;
+      }
+    p->ring_cap = cap;
+  }
+  if (bytes > p->meta_cap) {
+    CK(cudaDeviceSynchronize());
+    cudaFree(p->d_meta);
+    p->d_meta = nullptr;
+    size_t cap = std::max<size_t>(bytes, 4096);
+    if (cudaMalloc(&p->d_meta, cap) != cudaSuccess) {
+      p->meta_cap = 0;
+      return LOGMEL_ERR_OOM;
+    }
+    p->meta_cap = cap;
+  }
+  return LOGMEL_OK;
+}
+
+logmel_status logmel_compute(logmel_plan* p, const float* pcm, const int64_t* off, int64_t n_utt,
+                             float* out, void* stream) {
+  if (!p) return LOGMEL_ERR_INVALID_ARG;
+  logmel_status st = check_offsets(off, n_utt);
+  if (st != LOGMEL_OK) return st;
+  if (n_utt == 0) return LOGMEL_OK;
+  if (n_utt >= INT32_MAX) return LOGMEL_ERR_INPUT_TOO_LONG;
+  // frames and tiles per utterance (the ragged index map)
+  int64_t frames = 0, tiles = 0;
+  for (int64_t u = 0; u < n_utt; ++u) {
+    const int64_t f = frames_of(off[u + 1] - off[u]);
+    frames += f;
+    tiles += (f + TILE - 1) / TILE;
+  }
+  if (frames == 0) return LOGMEL_OK;
+  if (!pcm || !out) return LOGMEL_ERR_INVALID_ARG;
+  if (tiles >= INT32_MAX) return LOGMEL_ERR_INPUT_TOO_LONG;
+  const size_t bytes = meta_bytes(n_utt);
+  st = ensure_meta(p, bytes);
+  if (st != LOGMEL_OK) return st;
+  PinnedSlot& slot = p->ring[p->ring_next];
+  p->ring_next = (p->ring_next + 1) % RING;
+  if (slot.used) CK(cudaEventSynchronize(slot.done));
+  MetaView hv = meta_view(slot.host, n_utt);
+  hv.frame_off[0] = 0;
+  hv.tile_off[0] = 0;
+  for (int64_t u = 0; u <= n_utt; ++u) hv.sample_off[u] = off[u];
+  for (int64_t u = 0; u < n_utt; ++u) {
+    const int64_t f = frames_of(off[u + 1] - off[u]);
+    hv.frame_off[u + 1] = hv.frame_off[u] + f;
+    hv.tile_off[u + 1] = hv.tile_off[u] + (int)((f + TILE - 1) / TILE);
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  CK(cudaMemcpyAsync(p->d_meta, slot.host, bytes, cudaMemcpyHostToDevice, s));
+  CK(cudaEventRecord(slot.done, s));
+  slot.used = true;
+  MetaView dv = meta_view(p->d_meta, n_utt);
+  Args a{};
+  a.tables = p->d_tables;
+  a.out = out;
+  a.status = p->d_status;
+  a.mode = 0;
+  a.num_tiles = (int)tiles;
+  a.n_mels = p->n_mels;
+  a.pcm = pcm;
+  a.sample_off = dv.sample_off;
+  a.frame_off = dv.frame_off;
+  a.tile_off = dv.tile_off;
+  a.n_utt = (int)n_utt;
+  const int grid = (int)std::min<int64_t>(tiles, p->max_ctas);
+  CK(launch(p, a, grid, s));
+  return LOGMEL_OK;
+}
+
+// ---------------------------------------------------------------------------
+// streaming
+// ---------------------------------------------------------------------------
+logmel_status logmel_stream_create(logmel_plan* p, int n_streams, logmel_stream** out) {
+  if (!p || !out || n_streams < 1) return LOGMEL_ERR_INVALID_ARG;
+  *out = nullptr;
+  logmel_stream* st = new (std::nothrow) logmel_stream();
+  if (!st) return LOGMEL_ERR_OOM;
+  st->plan = p;
+  st->n_streams = n_streams;
+  st->total.assign(n_streams, 0);
+  st->carry_len.assign(n_streams, 0);
+  if (cudaMalloc(&st->d_carry, sizeof(float) * (size_t)n_streams * CARRY_CAP) != cudaSuccess ||
+      cudaMalloc(&st->d_carry_len, sizeof(int) * (size_t)n_streams) != cudaSuccess) {
+    logmel_stream_destroy(st);
+    return LOGMEL_ERR_OOM;
+  }
+  if (cudaMemset(st->d_carry, 0, sizeof(float) * (size_t)n_streams * CARRY_CAP) != cudaSuccess ||
+      cudaMemset(st->d_carry_len, 0, sizeof(int) * (size_t)n_streams) != cudaSuccess ||
+      cudaDeviceSynchronize() != cudaSuccess) {
+    logmel_stream_destroy(st);
+    return LOGMEL_ERR_CUDA;
+  }
+  *out = st;
+  return LOGMEL_OK;
+}
+
+void logmel_stream_destroy(logmel_stream* st) {
+  if (!st) return;
+  cudaDeviceSynchronize();
+  cudaFree(st->d_carry);
+  cudaFree(st->d_carry_len);
+  delete st;
+}
+
+int64_t logmel_stream_frames_for_push(const logmel_stream* st, int id, int64_t len) {
+  if (!st || id < 0 || id >= st->n_streams || len < 0) return -1;
+  return frames_of(st->carry_len[id] + len);
+}
+
+int64_t logmel_stream_max_frames(const logmel_stream* st, int64_t len) {
+  if (!st || len < 0) return -1;
+  int64_t mx = 0;
+  for (int s = 0; s < st->n_streams; ++s) mx = std::max(mx, frames_of(st->carry_len[s] + len));
+  return mx;
+}
+
+static logmel_status push_impl(logmel_stream* st, int base, int count, const float* chunks,
+                               int64_t chunk_stride, int64_t len, float* out, int64_t cap,
+                               int64_t* n_out, void* stream) {
+  logmel_plan* p = st->plan;
+  if (len < 0 || cap < 0 || !n_out) return LOGMEL_ERR_INVALID_ARG;
+  if (len > (int64_t)INT32_MAX / 2) return LOGMEL_ERR_INPUT_TOO_LONG;
+  int64_t max_n = 0;
+  for (int i = 0; i < count; ++i) max_n = std::max(max_n, frames_of(st->carry_len[base + i] + len));
+  if (max_n > cap) return LOGMEL_ERR_INVALID_ARG;
+  if (len > 0 && !chunks) return LOGMEL_ERR_INVALID_ARG;
+  if (max_n > 0 && !out) return LOGMEL_ERR_INVALID_ARG;
+  if (count > 1 && chunk_stride < len) return LOGMEL_ERR_INVALID_ARG;
+  const int spt = max_n <= TILE / 4 ? 4 : (max_n <= TILE / 2 ? 2 : 1);
+  const int64_t tps = max_n <= TILE ? 1 : (max_n + TILE - 1) / TILE;
+  const int64_t tiles = (int64_t)((count + spt - 1) / spt) * tps;
+  if (tiles >= INT32_MAX || (int64_t)count * cap >= ((int64_t)1 << 40)) return LOGMEL_ERR_INPUT_TOO_LONG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (len > 0) {
+    Args a{};
+    a.tables = p->d_tables;
+    a.out = out;
+    a.status = p->d_status;
+    a.mode = 1;
+    a.num_tiles = (int)tiles;
+    a.n_mels = p->n_mels;
+    a.carry = st->d_carry;
+    a.carry_len = st->d_carry_len;
+    a.chunks = chunks;
+    a.chunk_stride = chunk_stride;
+    a.push_len = len;
+    a.stream_base = base;
+    a.n_push_streams = count;
+    a.spt = spt;
+    a.tps = (int)tps;
+    a.update_carry = tps == 1 ? 1 : 0;
+    a.out_cap = cap;
+    const int grid = (int)std::min<int64_t>(tiles, p->max_ctas);
+    CK(launch(p, a, grid, s));
+    if (tps > 1) {
+      carry_update_kernel<<<count, 128, 0, s>>>(st->d_carry, st->d_carry_len, chunks, chunk_stride,
+                                                len, base);
+      CK(cudaGetLastError());
+    }
+  }
+  for (int i = 0; i < count; ++i) {
+    const int id = base + i;
+    const int64_t B = st->carry_len[id] + len;
+    const int64_t n = frames_of(B);
+    n_out[i] = n;
+    st->carry_len[id] = (int)(B - n * HOP);
+    st->total[id] += len;
+  }
+  return LOGMEL_OK;
+}
+
+logmel_status logmel_stream_push(logmel_stream* st, int id, const float* chunk, int64_t len,
+                                 float* out, int64_t cap, int64_t* n_out, void* stream) {
+  if (!st || id < 0 || id >= st->n_streams) return LOGMEL_ERR_INVALID_ARG;
+  return push_impl(st, id, 1, chunk, len, len, out, cap, n_out, stream);
+}
+
+logmel_status logmel_stream_push_batch(logmel_stream* st, const float* chunks, int64_t stride,
+                                       int64_t len, float* out, int64_t cap, int64_t* n_out,
+                                       void* stream) {
+  if (!st) return LOGMEL_ERR_INVALID_ARG;
+  return push_impl(st, 0, st->n_streams, chunks, stride, len, out, cap, n_out, stream);
+}
+
+struct StateHeader {
+  uint32_t magic;
+  int32_t n_streams;
+  int32_t carry_cap;
+  int32_t reserved;
+};
+
+int64_t logmel_stream_state_bytes(const logmel_stream* st) {
+  if (!st) return -1;
+  return (int64_t)sizeof(StateHeader) +
+         (int64_t)st->n_streams * (int64_t)(sizeof(int64_t) + sizeof(int32_t) + 4 * CARRY_CAP);
+}
+
+logmel_status logmel_stream_get_state(logmel_stream* st, void* blob, int64_t bytes, void* stream) {
+  if (!st || !blob || bytes != logmel_stream_state_bytes(st)) return LOGMEL_ERR_INVALID_ARG;
+  const int S = st->n_streams;
+  std::vector<float> carry((size_t)S * CARRY_CAP);
+  std::vector<int> lens(S);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  CK(cudaMemcpyAsync(carry.data(), st->d_carry, carry.size() * 4, cudaMemcpyDeviceToHost, s));
+  CK(cudaMemcpyAsync(lens.data(), st->d_carry_len, (size_t)S * 4, cudaMemcpyDeviceToHost, s));
+  CK(cudaStreamSynchronize(s));
+  for (int i = 0; i < S; ++i)
+    if (lens[i] != st->carry_len[i]) return LOGMEL_ERR_DEVICE_STATUS;
+  unsigned char* b = static_cast<unsigned char*>(blob);
+  StateHeader h{STATE_MAGIC, S, CARRY_CAP, 0};
+  std::memcpy(b, &h, sizeof h);
+  b += sizeof h;
+  for (int i = 0; i < S; ++i) {
+    std::memcpy(b, &st->total[i], 8);
+    std::memcpy(b + 8, &lens[i], 4);
+    std::memcpy(b + 12, &carry[(size_t)i * CARRY_CAP], 4 * CARRY_CAP);
+    b += 12 + 4 * CARRY_CAP;
+  }
+  return LOGMEL_OK;
+}
+
+logmel_status logmel_stream_set_state(logmel_stream* st, const void* blob, int64_t bytes,
+                                      void* stream) {
+  if (!st || !blob || bytes != logmel_stream_state_bytes(st)) return LOGMEL_ERR_INVALID_ARG;
+  const unsigned char* b = static_cast<const unsigned char*>(blob);
+  StateHeader h;
+  std::memcpy(&h, b, sizeof h);
+  if (h.magic != STATE_MAGIC || h.n_streams != st->n_streams || h.carry_cap != CARRY_CAP)
+    return LOGMEL_ERR_INVALID_ARG;
+  b += sizeof h;
+  const int S = st->n_streams;
+  std::vector<float> carry((size_t)S * CARRY_CAP);
+  std::vector<int> lens(S);
+  std::vector<int64_t> total(S);
+  for (int i = 0; i < S; ++i) {
+    std::memcpy(&total[i], b, 8);
+    std::memcpy(&lens[i], b + 8, 4);
+    std::memcpy(&carry[(size_t)i * CARRY_CAP], b + 12, 4 * CARRY_CAP);
+    b += 12 + 4 * CARRY_CAP;
+    const int64_t expect = total[i] - frames_of(total[i]) * HOP;
+    if (total[i] < 0 || lens[i] != expect) return LOGMEL_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  CK(cudaMemcpyAsync(st->d_carry, carry.data(), carry.size() * 4, cudaMemcpyHostToDevice, s));
+  CK(cudaMemcpyAsync(st->d_carry_len, lens.data(), (size_t)S * 4, cudaMemcpyHostToDevice, s));
+  CK(cudaStreamSynchronize(s));
+  st->total = total;
+  st->carry_len = lens;
+  return LOGMEL_OK;
+}
+
+logmel_status logmel_stream_reset(logmel_stream* st, int id, void* stream) {
+  if (!st || id >= st->n_streams) return LOGMEL_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (id < 0) {
+    CK(cudaMemsetAsync(st->d_carry_len, 0, sizeof(int) * (size_t)st->n_streams, s));
+    std::fill(st->total.begin(), st->total.end(), 0);
+    std::fill(st->carry_len.begin(), st->carry_len.end(), 0);
+  } else {
+    CK(cudaMemsetAsync(st->d_carry_len + id, 0, sizeof(int), s));
+    st->total[id] = 0;
+    st->carry_len[id] = 0;
+  }
+  return LOGMEL_OK;
+}
+
+logmel_status logmel_plan_device_status(logmel_plan* p, int* code, void* stream) {
+  if (!p || !code) return LOGMEL_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int v = 0;
+  CK(cudaMemcpyAsync(&v, p->d_status, sizeof(int), cudaMemcpyDeviceToHost, s));
+  CK(cudaMemsetAsync(p->d_status, 0, sizeof(int), s));
+  CK(cudaStreamSynchronize(s));
+  *code = v;
+  return LOGMEL_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,590 @@
+// Fused log-mel kernel for sm_100a.
+//
+// Computes, per frame, the pipeline of "从零理解 ASR：音频基础、Qwen3-ASR 架构，
+// 以及离线 vs 流式推理原理", section 2.3 steps 1-5: 400-sample frame every 160
+// samples -> symmetric Hamming window -> real DFT (201 bins) -> |X|^2 ->
+// 128 triangular mel filters -> ln(max(., 1e-10)).
+//
+// Structure (one persistent kernel, 160 threads, tiles of 32 frames; frame
+// slots d and d + 16 form the pair carried by one thread):
+//   stage   each tile's overlapping sample span is copied from HBM once into
+//           shared memory with cp.async, 162 floats per 160-sample hop block
+//           (the 2 pad floats make pass A's reads bank-conflict free)
+//   pass A  real FFT-400 as a complex FFT-200 of z[m] = x[2m] + i x[2m+1]
+//           (window applied on load), Cooley-Tukey 200 = 20 x 10: ten
+//           20-point DFTs per frame (prime-factor 4 x 5, no inner twiddles),
+//           then the twiddle e^{-2 pi i m2 k1 / 200}
+//   pass B  twenty 10-point DFTs (prime-factor 2 x 5); a thread owns the two
+//           tasks k1 and 20 - k1, so Z[k] and Z[200 - k] meet in registers and
+//           the real-FFT split X[k] = (A + u_k B) / 2, u_k = -i e^{-2 pi i k/400},
+//           and the power |2 X[k]|^2 need no exchange
+//   mel     lane = frame, warp = group of bands balanced by nonzeros; each
+//           band sums weight * power over its contiguous bins in a fixed order
+//           (fully unrolled for the default 128-band filterbank, weights read
+//           from the kernel's constant parameter bank)
+//   log     ln via __logf, exact floor constant when the energy is < 1e-10
+//   store   coalesced rows of n_mels fp32
+// Two frames ride in the two lanes of packed f32x2 arithmetic (add/sub/mul/
+// fma .f32x2), so a frame's arithmetic never depends on its partner frame:
+// a frame gives the same bits whichever tile, slot or partner it lands in,
+// which is what makes streaming output equal offline output bit for bit.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "mel_layout_default.h"
+
+namespace logmel {
+
+constexpr int NFFT = 400;
+constexpr int NBINS = NFFT / 2 + 1;   // 201
+constexpr int HOP = 160;
+constexpr int TILE = 32;              // frames per tile
+constexpr int DUOS = TILE / 2;        // frame pairs carried by f32x2 lanes
+constexpr int N1 = 20;                // FFT-200 = N1 x N2, m = N2*m1 + m2, k = k1 + N1*k2
+constexpr int N2 = 10;
+constexpr int ROLES = 10;             // threads per frame pair in each pass
+constexpr int THREADS = DUOS * ROLES; // 160
+constexpr int BLK = 162;              // smem floats per hop block (160 + 2 pad)
+constexpr int SPAN_BLOCKS = 44;       // >= sum over groups of (frames + 3)
+constexpr int PSTRIDE = NBINS - 2;    // power rows hold bins 1..199 (odd stride: conflict-free)
+constexpr int YROW = N2;              // float4 per pass-A output row
+constexpr int YDUO = N1 * YROW + 1;   // float4 per frame pair (odd: conflict-free by lane = pair)
+constexpr int MAX_GROUPS = 4;
+constexpr int MEL_WARPS = THREADS / 32;   // 5
+constexpr int MAX_MELS = NBINS;
+constexpr int MAX_WEIGHTS = 2 * NBINS;    // each bin feeds at most two triangles
+constexpr int OSTRIDE = TILE + 1;         // staged output [n_mels][33]
+constexpr int CARRY_CAP = NFFT;           // carried samples per stream (< 400)
+
+// ln(1e-10) rounded to fp32: the value written wherever the mel energy is
+// below 1e-10 (section 2.3 step 5's floor).
+constexpr float LOG_FLOOR = -23.025850929940457f;
+constexpr float ENERGY_FLOOR = 1e-10f;
+
+// Constant tables, built in float64 on the host by the plan and rounded to fp32.
+struct __align__(16) Tables {
+  float2 win[N2][N1];          // (w[20 m1 + 2 m2], w[20 m1 + 2 m2 + 1]) at [m2][m1]
+  float4 tw[N2][N1];           // (c, c, s, s): e^{-2 pi i m2 k1 / 200} = c - i s
+  float2 twn[N2][N1];          // (-s, -s)
+  float4 post[NFFT / 2];       // (ur, ur, ui, ui): u_k = -i e^{-2 pi i k / 400}
+  float2 postn[NFFT / 2];      // (-ui, -ui)
+};
+
+// One contiguous run of a tile's frames taken from one source signal.
+// The source is the concatenation src0[0 .. len0) ++ src1[...] (offline:
+// an utterance; streaming: carry ++ pushed chunk).
+struct Group {
+  const float* src0;
+  const float* src1;
+  int64_t len0;
+  int64_t start;      // first staged position (160 * first frame)
+  int64_t out_row;    // output row of the group's first frame
+  int nstage;         // samples staged from `start`
+  int nframes;
+  int slot0;          // first frame slot of the group in the tile
+  int block0;         // first hop block of the group's span in shared memory
+  // streaming carry update (carry_len_dst == nullptr: none)
+  float* carry_dst;
+  int* carry_len_dst;
+  int new_carry_len;
+  int carry_from;     // span-relative position of the new carry's first sample
+};
+
+struct Args {
+  const Tables* tables;
+  float* out;
+  int* status;
+  int mode;             // 0: offline ragged batch, 1: streaming push
+  int num_tiles;
+  int n_mels;
+  // offline
+  const float* pcm;
+  const int64_t* sample_off;   // [n_utt + 1]
+  const int64_t* frame_off;    // [n_utt + 1]
+  const int* tile_off;         // [n_utt + 1]
+  int n_utt;
+  // streaming
+  float* carry;                // [n_streams][CARRY_CAP]
+  int* carry_len;              // [n_streams]
+  const float* chunks;
+  int64_t chunk_stride;
+  int64_t push_len;
+  int stream_base;
+  int n_push_streams;
+  int spt;                     // streams per tile (1, 2, 4)
+  int tps;                     // tiles per stream
+  int update_carry;            // 1: this kernel writes the new carries
+  int64_t out_cap;             // output rows per stream
+  // filterbank (per plan): weights / 4 (the real split yields |2 X|^2), and
+  // for the generic (non-default) layout the band structure
+  float mel_w[MAX_WEIGHTS];
+  short mel_lo[MAX_MELS];      // first nonzero bin
+  short mel_cnt[MAX_MELS];     // contiguous nonzero bins
+  short mel_woff[MAX_MELS];    // offset into mel_w
+  short warp_band[MEL_WARPS + 1];
+};
+
+enum DeviceStatus : int { STATUS_OK = 0, STATUS_SPAN_OVERFLOW = 1, STATUS_SLOT_OVERFLOW = 2 };
+
+// ---------------------------------------------------------------------------
+// packed fp32 pair arithmetic (sm_100a .f32x2): lane x = frame A, lane y = frame B
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  unsigned long long ua, ub, ud;
+  ua = *reinterpret_cast<unsigned long long*>(&a);
+  ub = *reinterpret_cast<unsigned long long*>(&b);
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(ud) : "l"(ua), "l"(ub));
+  return *reinterpret_cast<float2*>(&ud);
+}
+__device__ __forceinline__ float2 bcast(float c) { return make_float2(c, c); }
+
+struct cx {
+  float2 re, im;
+};
+
+// 2-point DFT in place.
+__device__ __forceinline__ void dft2(cx& a, cx& b) {
+  cx s{add2(a.re, b.re), add2(a.im, b.im)};
+  cx d{sub2(a.re, b.re), sub2(a.im, b.im)};
+  a = s;
+  b = d;
+}
+
+// 4-point forward DFT in place (X1 = d02 - i d13, X3 = d02 + i d13).
+__device__ __forceinline__ void dft4(cx& a0, cx& a1, cx& a2, cx& a3) {
+  float2 s02r = add2(a0.re, a2.re), s02i = add2(a0.im, a2.im);
+  float2 d02r = sub2(a0.re, a2.re), d02i = sub2(a0.im, a2.im);
+  float2 s13r = add2(a1.re, a3.re), s13i = add2(a1.im, a3.im);
+  float2 d13r = sub2(a1.re, a3.re), d13i = sub2(a1.im, a3.im);
+  a0 = cx{add2(s02r, s13r), add2(s02i, s13i)};
+  a2 = cx{sub2(s02r, s13r), sub2(s02i, s13i)};
+  a1 = cx{add2(d02r, d13i), sub2(d02i, d13r)};
+  a3 = cx{sub2(d02r, d13i), add2(d02i, d13r)};
+}
+
+// 5-point forward DFT in place: with t1 = x1 + x4, t2 = x2 + x3, t3 = x1 - x4,
+// t4 = x2 - x3 and c_j = cos(2 pi j / 5), s_j = sin(2 pi j / 5):
+// X1,4 = (x0 + c1 t1 + c2 t2) -/+ i (s1 t3 + s2 t4),
+// X2,3 = (x0 + c2 t1 + c1 t2) -/+ i (s2 t3 - s1 t4).
+__device__ __forceinline__ void dft5(cx& x0, cx& x1, cx& x2, cx& x3, cx& x4) {
+  const float2 C1 = bcast(0.30901699437494745f), C2 = bcast(-0.80901699437494745f);
+  const float2 S1 = bcast(0.95105651629515353f), S2 = bcast(0.58778525229247314f);
+  const float2 NS1 = bcast(-0.95105651629515353f);
+  float2 t1r = add2(x1.re, x4.re), t1i = add2(x1.im, x4.im);
+  float2 t2r = add2(x2.re, x3.re), t2i = add2(x2.im, x3.im);
+  float2 t3r = sub2(x1.re, x4.re), t3i = sub2(x1.im, x4.im);
+  float2 t4r = sub2(x2.re, x3.re), t4i = sub2(x2.im, x3.im);
+  float2 a1r = fma2(t2r, C2, fma2(t1r, C1, x0.re)), a1i = fma2(t2i, C2, fma2(t1i, C1, x0.im));
+  float2 a2r = fma2(t2r, C1, fma2(t1r, C2, x0.re)), a2i = fma2(t2i, C1, fma2(t1i, C2, x0.im));
+  float2 b1r = fma2(t4r, S2, mul2(t3r, S1)), b1i = fma2(t4i, S2, mul2(t3i, S1));
+  float2 b2r = fma2(t4r, NS1, mul2(t3r, S2)), b2i = fma2(t4i, NS1, mul2(t3i, S2));
+  x0 = cx{add2(add2(x0.re, t1r), t2r), add2(add2(x0.im, t1i), t2i)};
+  x1 = cx{add2(a1r, b1i), sub2(a1i, b1r)};
+  x4 = cx{sub2(a1r, b1i), add2(a1i, b1r)};
+  x2 = cx{add2(a2r, b2i), sub2(a2i, b2r)};
+  x3 = cx{sub2(a2r, b2i), add2(a2i, b2r)};
+}
+
+// Prime-factor 20 = 4 x 5 (Good-Thomas): input n = (5 n1 + 4 n2) mod 20 sits at
+// register n; afterwards X[q] sits at register pos20(q) = (5 (q%4) + 4 (q%5)) mod 20.
+__host__ __device__ constexpr int pos20(int q) { return (5 * (q % 4) + 4 * (q % 5)) % 20; }
+__device__ __forceinline__ void dft20(cx (&x)[20]) {
+#pragma unroll
+  for (int n2 = 0; n2 < 5; ++n2)
+    dft4(x[(4 * n2) % 20], x[(5 + 4 * n2) % 20], x[(10 + 4 * n2) % 20], x[(15 + 4 * n2) % 20]);
+#pragma unroll
+  for (int k1 = 0; k1 < 4; ++k1)
+    dft5(x[(5 * k1) % 20], x[(5 * k1 + 4) % 20], x[(5 * k1 + 8) % 20], x[(5 * k1 + 12) % 20],
+         x[(5 * k1 + 16) % 20]);
+}
+
+// Prime-factor 10 = 2 x 5: input n = (5 n1 + 2 n2) mod 10 at register n;
+// afterwards X[q] sits at register pos10(q) = (5 (q%2) + 2 (q%5)) mod 10.
+__host__ __device__ constexpr int pos10(int q) { return (5 * (q % 2) + 2 * (q % 5)) % 10; }
+__device__ __forceinline__ void dft10(cx (&x)[10]) {
+#pragma unroll
+  for (int n2 = 0; n2 < 5; ++n2) dft2(x[(2 * n2) % 10], x[(5 + 2 * n2) % 10]);
+#pragma unroll
+  for (int k1 = 0; k1 < 2; ++k1)
+    dft5(x[(5 * k1) % 10], x[(5 * k1 + 2) % 10], x[(5 * k1 + 4) % 10], x[(5 * k1 + 6) % 10],
+         x[(5 * k1 + 8) % 10]);
+}
+
+__device__ __forceinline__ cx sel(bool p, const cx& a, const cx& b) {
+  return p ? a : b;
+}
+
+// ---------------------------------------------------------------------------
+// shared memory layout
+// ---------------------------------------------------------------------------
+struct __align__(16) Smem {
+  Tables tab;
+  float4 y[DUOS * YDUO];                 // pass A -> pass B; later the staged output
+  float span[SPAN_BLOCKS * BLK];         // staged samples; later the power spectra
+  Group groups[MAX_GROUPS];
+  int64_t slot_row[TILE];
+  int slot_block[TILE];
+  int ngroups;
+  int nslots;
+};
+static_assert(MAX_MELS * OSTRIDE <= DUOS * YDUO * 4, "staged output must fit the pass buffer");
+static_assert(TILE * PSTRIDE <= SPAN_BLOCKS * BLK, "power buffer must fit the span buffer");
+static_assert(sizeof(mel_default::WARP_BAND) == sizeof(int) * (MEL_WARPS + 1), "default band split must match the mel warps");
+static_assert(sizeof(Tables) % 16 == 0, "tables are copied as float4");
+
+// Ampere-style asynchronous global -> shared copies (4 or 8 bytes, L1-allocating).
+__device__ __forceinline__ void cp_async4(float* dst, const float* src) {
+  const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(dst));
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async8(float* dst, const float* src) {
+  const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(dst));
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
+}
+
+__device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+__device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
+
+__device__ __forceinline__ float src_at(const Group& g, int64_t pos) {
+  return pos < g.len0 ? g.src0[pos] : g.src1[pos - g.len0];
+}
+
+// Thread 0: the tile's groups (sources, frames, span blocks, output rows).
+__device__ void setup_tile(Smem& S, const Args& a, int tile) {
+  int ng = 0, slot = 0, block = 0;
+  if (a.mode == 0) {
+    int lo = 0, hi = a.n_utt - 1;   // last u with tile_off[u] <= tile
+    while (lo < hi) {
+      int mid = (lo + hi + 1) >> 1;
+      if (a.tile_off[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    const int u = lo;
+    const int64_t f0 = (int64_t)(tile - a.tile_off[u]) * TILE;
+    const int64_t nfr = a.frame_off[u + 1] - a.frame_off[u];
+    const int cnt = (int)min64(TILE, nfr - f0);
+    Group& g = S.groups[0];
+    g.src0 = a.pcm + a.sample_off[u];
+    g.src1 = nullptr;
+    g.len0 = a.sample_off[u + 1] - a.sample_off[u];
+    g.start = f0 * HOP;
+    g.out_row = a.frame_off[u] + f0;
+    g.nframes = cnt;
+    g.nstage = cnt > 0 ? HOP * (cnt - 1) + NFFT : 0;
+    g.slot0 = 0;
+    g.block0 = 0;
+    g.carry_len_dst = nullptr;
+    ng = 1;
+    slot = cnt;
+    block = (g.nstage + HOP - 1) / HOP;
+  } else {
+    const int sg = tile / a.tps, st = tile - sg * a.tps;
+    for (int j = 0; j < a.spt; ++j) {
+      const int sl = sg * a.spt + j;
+      if (sl >= a.n_push_streams) break;
+      const int s = a.stream_base + sl;
+      const int c = a.carry_len[s];
+      const int64_t B = c + a.push_len;
+      const int64_t n = B >= NFFT ? (B - NFFT) / HOP + 1 : 0;
+      const int64_t f0 = (int64_t)st * TILE;
+      const int cnt = (int)max64(0, min64(TILE / a.spt, n - f0));
+      const bool owner = (st == 0) && a.update_carry;
+      if (cnt == 0 && !owner) continue;
+      Group& g = S.groups[ng];
+      g.src0 = a.carry + (int64_t)s * CARRY_CAP;
+      g.src1 = a.chunks + (int64_t)sl * a.chunk_stride;
+      g.len0 = c;
+      g.start = f0 * HOP;
+      const int64_t end = min64(B, g.start + (int64_t)HOP * cnt + NFFT);
+      g.nstage = (int)max64(0, end - g.start);
+      g.nframes = cnt;
+      g.slot0 = slot;
+      g.block0 = block;
+      g.out_row = (int64_t)sl * a.out_cap + f0;
+      g.carry_len_dst = nullptr;
+      if (owner) {
+        g.carry_dst = a.carry + (int64_t)s * CARRY_CAP;
+        g.carry_len_dst = a.carry_len + s;
+        g.new_carry_len = (int)(B - n * HOP);
+        g.carry_from = (int)(n * HOP - g.start);
+      }
+      ++ng;
+      slot += cnt;
+      block += (g.nstage + HOP - 1) / HOP;
+    }
+  }
+  if (block > SPAN_BLOCKS || slot > TILE) {
+    atomicExch(a.status, block > SPAN_BLOCKS ? STATUS_SPAN_OVERFLOW : STATUS_SLOT_OVERFLOW);
+    ng = 0;
+    slot = 0;
+  }
+  S.ngroups = ng;
+  S.nslots = slot;
+}
+
+// ---------------------------------------------------------------------------
+// mel stage: lane = frame slot s, P = that frame's power row (bins 1..199 at
+// P[k - 1]), o = staged output [band][OSTRIDE]
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float log_floor(float acc) {
+  return acc < ENERGY_FLOOR ? LOG_FLOOR : __logf(acc);
+}
+
+// Default 128-band layout, unrolled at compile time: bins and weight offsets
+// are constants, the weights come from the constant parameter bank.
+template <int M, int MEND>
+struct MelBands {
+  static __device__ __forceinline__ void run(const float* P, float* o, int s, const float* w) {
+    if constexpr (M < MEND) {
+      constexpr int lo = mel_default::LO[M], cnt = mel_default::CNT[M], wo = mel_default::WOFF[M];
+      float acc = 0.f;
+#pragma unroll
+      for (int j = 0; j < cnt; ++j) acc = fmaf(w[wo + j], P[lo + j], acc);
+      o[M * OSTRIDE + s] = log_floor(acc);
+      MelBands<M + 1, MEND>::run(P, o, s, w);
+    }
+  }
+};
+
+template <int W>
+__device__ __forceinline__ void mel_default_warp(const float* P, float* o, int s, const float* w) {
+  MelBands<mel_default::WARP_BAND[W], mel_default::WARP_BAND[W + 1]>::run(P, o, s, w);
+}
+
+__device__ __forceinline__ void mel_generic_warp(const Args& a, int w, const float* P, float* o, int s) {
+  const int mb = a.warp_band[w], me = a.warp_band[w + 1];
+  for (int m = mb; m < me; ++m) {
+    const int lo = a.mel_lo[m], cnt = a.mel_cnt[m], wo = a.mel_woff[m];
+    float acc = 0.f;
+    for (int j = 0; j < cnt; ++j) acc = fmaf(a.mel_w[wo + j], P[lo + j], acc);
+    o[m * OSTRIDE + s] = log_floor(acc);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// pass B real split for one pair slot: Z[k] (zk) and Z[200 - k] (zm) ->
+// |2 X[k]|^2 and |2 X[200 - k]|^2 for the two frames of the pair
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void split_power(const Smem& S, const cx& zk, const cx& zm, int k,
+                                            float2& pk, float2& pm) {
+  const float2 Ar = add2(zk.re, zm.re), Ai = sub2(zk.im, zm.im);   // A = Z[k] + conj Z[-k]
+  const float2 Br = sub2(zk.re, zm.re), Bi = add2(zk.im, zm.im);   // B = Z[k] - conj Z[-k]
+  const float4 u = S.tab.post[k];
+  const float2 nui = S.tab.postn[k];
+  const float2 ur = make_float2(u.x, u.y), ui = make_float2(u.z, u.w);
+  const float2 Tr = fma2(Bi, nui, mul2(Br, ur));                    // T = u_k B
+  const float2 Ti = fma2(Br, ui, mul2(Bi, ur));
+  const float2 pr = add2(Ar, Tr), pi = add2(Ai, Ti);                // 2 X[k]
+  const float2 qr = sub2(Ar, Tr), qi = sub2(Ai, Ti);                // 2 conj X[200 - k]
+  pk = fma2(pi, pi, mul2(pr, pr));
+  pm = fma2(qi, qi, mul2(qr, qr));
+}
+
+template <bool kDefaultMel>
+__global__ void __launch_bounds__(THREADS, 2) logmel_fused_kernel(const __grid_constant__ Args a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  Smem& S = *reinterpret_cast<Smem*>(smem_raw);
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int half = lane >> 4, d = lane & 15;       // frame pair d = slots (d, d + 16)
+  const int role = 2 * warp + half;               // pass A: m2; pass B: k1 pair index
+
+  {  // constant tables -> shared memory, once per CTA
+    const float4* src = reinterpret_cast<const float4*>(a.tables);
+    float4* dst = reinterpret_cast<float4*>(&S.tab);
+    for (int i = tid; i < (int)(sizeof(Tables) / 16); i += THREADS) dst[i] = src[i];
+  }
+
+  const int n_mels = a.n_mels;
+  for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
+    __syncthreads();   // previous tile fully written out; tables visible
+    if (tid == 0) setup_tile(S, a, tile);
+    __syncthreads();
+    const int ng = S.ngroups;
+
+    // ---- stage: each group's span -> hop blocks of BLK floats ---------------
+    // cp.async puts every load of the span in flight at once (no register
+    // round trip); 8-byte copies when the source is 8-byte aligned.
+    for (int gi = 0; gi < ng; ++gi) {
+      const Group& g = S.groups[gi];
+      float* dst = S.span + g.block0 * BLK;
+      const float* base = g.src0 + g.start;
+      if (g.src1 == nullptr && (reinterpret_cast<uintptr_t>(base) & 7) == 0 && (g.nstage & 1) == 0) {
+        for (int i = 2 * tid; i < g.nstage; i += 2 * THREADS) {
+          const int b = i / HOP;
+          cp_async8(dst + b * BLK + (i - b * HOP), base + i);
+        }
+      } else {
+        for (int i = tid; i < g.nstage; i += THREADS) {
+          const int64_t pos = g.start + i;
+          const float* src = pos < g.len0 ? g.src0 + pos : g.src1 + (pos - g.len0);
+          const int b = i / HOP;
+          cp_async4(dst + b * BLK + (i - b * HOP), src);
+        }
+      }
+    }
+    if (tid < TILE) {  // per-slot span block and output row
+      int blk = 0;
+      int64_t row = -1;
+      for (int gi = 0; gi < ng; ++gi) {
+        const Group& g = S.groups[gi];
+        if (tid >= g.slot0 && tid < g.slot0 + g.nframes) {
+          blk = g.block0 + (tid - g.slot0);
+          row = g.out_row + (tid - g.slot0);
+        }
+      }
+      S.slot_block[tid] = blk;
+      S.slot_row[tid] = row;
+    }
+    cp_async_wait_all();
+    __syncthreads();
+
+    // ---- streaming: write each owned stream's new carry from the span -----
+    for (int gi = 0; gi < ng; ++gi) {
+      const Group& g = S.groups[gi];
+      if (g.carry_len_dst == nullptr) continue;
+      const float* src = S.span + g.block0 * BLK;
+      for (int i = tid; i < g.new_carry_len; i += THREADS) {
+        const int p = g.carry_from + i;
+        const int b = p / HOP;
+        g.carry_dst[i] = src[b * BLK + (p - b * HOP)];
+      }
+      if (tid == 0) *g.carry_len_dst = g.new_carry_len;
+    }
+
+    // ---- pass A: window, 20-point DFTs over m1, twiddle --------------------
+    {
+      const int m2 = role;
+      const float* sa = S.span + BLK * S.slot_block[d] + 2 * m2;
+      const float* sb = S.span + BLK * S.slot_block[d + DUOS] + 2 * m2;
+      cx z[N1];
+#pragma unroll
+      for (int m1 = 0; m1 < N1; ++m1) {
+        const int off = BLK * (m1 / 8) + 20 * (m1 % 8);   // sample n = 20 m1 + 2 m2
+        const float2 xa = *reinterpret_cast<const float2*>(sa + off);
+        const float2 xb = *reinterpret_cast<const float2*>(sb + off);
+        const float2 w = S.tab.win[m2][m1];
+        z[m1].re = make_float2(xa.x * w.x, xb.x * w.x);
+        z[m1].im = make_float2(xa.y * w.y, xb.y * w.y);
+      }
+      dft20(z);
+      float4* yrow = S.y + d * YDUO + m2;
+#pragma unroll
+      for (int k1 = 0; k1 < N1; ++k1) {
+        cx v = z[pos20(k1)];
+        if (k1 > 0) {
+          const float4 t = S.tab.tw[m2][k1];
+          const float2 ns = S.tab.twn[m2][k1];
+          const float2 c = make_float2(t.x, t.y), sn = make_float2(t.z, t.w);
+          // (re + i im)(c - i s) = (re c + im s) + i (im c - re s)
+          const float2 re = fma2(v.im, sn, mul2(v.re, c));
+          const float2 im = fma2(v.re, ns, mul2(v.im, c));
+          v.re = re;
+          v.im = im;
+        }
+        yrow[k1 * YROW] = make_float4(v.re.x, v.re.y, v.im.x, v.im.y);
+      }
+    }
+    __syncthreads();
+
+    // ---- pass B: 10-point DFTs over m2, real split, power -----------------
+    {
+      const int r = role;
+      const bool r0 = (r == 0);
+      const int ka = r, kb = r0 ? 10 : N1 - r;
+      cx za[N2], zb[N2];
+      const float4* ya = S.y + d * YDUO + ka * YROW;
+      const float4* yb = S.y + d * YDUO + kb * YROW;
+#pragma unroll
+      for (int m2 = 0; m2 < N2; ++m2) {
+        const float4 va = ya[m2], vb = yb[m2];
+        za[m2] = cx{make_float2(va.x, va.y), make_float2(va.z, va.w)};
+        zb[m2] = cx{make_float2(vb.x, vb.y), make_float2(vb.z, vb.w)};
+      }
+      dft10(za);
+      dft10(zb);
+      // za[pos10(k2)] = Z[ka + 20 k2], zb[pos10(k2)] = Z[kb + 20 k2].
+      float* PA = S.span + d * PSTRIDE - 1;            // frame slot d, bin k at PA[k]
+      float* PB = S.span + (d + DUOS) * PSTRIDE - 1;   // frame slot d + 16
+      if (warp != 0) {
+        // roles 2..9: slot j couples Z[k], k = r + 20 j, with Z[200 - k] = zb[9 - j]
+#pragma unroll
+        for (int j = 0; j < N2; ++j) {
+          const int k = r + 20 * j;
+          float2 pk, pm;
+          split_power(S, za[pos10(j)], zb[pos10(9 - j)], k, pk, pm);
+          PA[k] = pk.x;
+          PB[k] = pk.y;
+          PA[200 - k] = pm.x;
+          PB[200 - k] = pm.y;
+        }
+      } else {
+        // roles 0 and 1 share this warp; role 0 owns the self-paired tasks
+        // k1 = 0 and 10: j < 5: k = 20 j with Z[200 - k] = za[(10 - j) % 10];
+        // j >= 5: k = 10 + 20 (j - 5) from zb[j - 5] with partner zb[14 - j];
+        // bin 100 (2 X[100] = 2 conj Z[100]) alone from za[5].  Bins 0 and
+        // 200 carry no filter weight and are not stored.
+#pragma unroll
+        for (int j = 0; j < N2; ++j) {
+          const cx zk = (j < 5) ? za[pos10(j)] : sel(r0, zb[pos10(j - 5)], za[pos10(j)]);
+          const cx zm = (j < 5) ? sel(r0, za[pos10((10 - j) % 10)], zb[pos10(9 - j)])
+                                : sel(r0, zb[pos10(14 - j)], zb[pos10(9 - j)]);
+          const int k = r0 ? (j < 5 ? 20 * j : 10 + 20 * (j - 5)) : r + 20 * j;
+          float2 pk, pm;
+          split_power(S, zk, zm, k, pk, pm);
+          if (k > 0) {
+            PA[k] = pk.x;
+            PB[k] = pk.y;
+            PA[200 - k] = pm.x;
+            PB[200 - k] = pm.y;
+          }
+        }
+        if (r0) {
+          const cx z = za[pos10(5)];
+          const float2 tr = add2(z.re, z.re), ti = add2(z.im, z.im);
+          const float2 p = fma2(ti, ti, mul2(tr, tr));
+          PA[100] = p.x;
+          PB[100] = p.y;
+        }
+      }
+    }
+    __syncthreads();
+
+    // ---- mel + log: warp = band group, lane = frame slot ------------------
+    {
+      const float* P = S.span + lane * PSTRIDE - 1;
+      float* o = reinterpret_cast<float*>(S.y);
+      if constexpr (kDefaultMel) {
+        switch (warp) {
+          case 0: mel_default_warp<0>(P, o, lane, a.mel_w); break;
+          case 1: mel_default_warp<1>(P, o, lane, a.mel_w); break;
+          case 2: mel_default_warp<2>(P, o, lane, a.mel_w); break;
+          case 3: mel_default_warp<3>(P, o, lane, a.mel_w); break;
+          default: mel_default_warp<4>(P, o, lane, a.mel_w); break;
+        }
+      } else {
+        mel_generic_warp(a, warp, P, o, lane);
+      }
+    }
+    __syncthreads();
+
+    // ---- store: rows of n_mels fp32, one warp per row ---------------------
+    {
+      const float* o = reinterpret_cast<const float*>(S.y);
+      const int ns = S.nslots;
+      for (int s = warp; s < ns; s += MEL_WARPS) {
+        float* row = a.out + S.slot_row[s] * n_mels;
+        for (int m = lane; m < n_mels; m += 32) row[m] = o[m * OSTRIDE + s];
+      }
+    }
+  }
+}
+
+}  // namespace logmel

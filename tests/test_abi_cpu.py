@@ -1,0 +1,82 @@
+"""The C-ABI library loads and exports every entry point include/logmel.h
+declares; argument checks that precede any CUDA call work without a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "logmel.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(logmel_[a-z_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def cdll():
+    from log_mel_spectrogram_logmel_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for required in ("logmel_plan_create", "logmel_plan_destroy", "logmel_num_frames",
+                     "logmel_frame_offsets", "logmel_compute", "logmel_stream_create",
+                     "logmel_stream_push", "logmel_stream_push_batch", "logmel_stream_get_state",
+                     "logmel_stream_set_state", "logmel_stream_destroy", "logmel_status_string"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(cdll):
+    missing = [n for n in _declared() if not hasattr(cdll, n)]
+    assert not missing, missing
+
+
+def test_binding_wraps_every_declared_symbol():
+    import log_mel_spectrogram_logmel_b200 as lm
+    assert lm.exported_symbols() == _declared()
+
+
+def test_status_strings(cdll):
+    f = cdll.logmel_status_string
+    f.restype = ctypes.c_char_p
+    f.argtypes = [ctypes.c_int]
+    assert f(0) == b"ok"
+    for code in range(1, 7):
+        assert f(code) and f(code) != b"unknown status"
+    assert f(99) == b"unknown status"
+
+
+def test_plan_argument_checks_precede_cuda(cdll):
+    create = cdll.logmel_plan_create
+    create.restype = ctypes.c_int
+    create.argtypes = [ctypes.c_int] * 4 + [ctypes.c_float] * 2 + [ctypes.POINTER(ctypes.c_void_p)]
+    h = ctypes.c_void_p()
+    assert create(16000, 512, 160, 128, 0.0, 8000.0, ctypes.byref(h)) == 2      # n_fft != 400
+    assert create(16000, 400, 100, 128, 0.0, 8000.0, ctypes.byref(h)) == 2      # hop != 160
+    assert create(16000, 400, 160, 202, 0.0, 8000.0, ctypes.byref(h)) == 2      # n_mels > 201
+    assert create(16000, 400, 160, 128, 0.0, 9000.0, ctypes.byref(h)) == 1      # fmax > sr / 2
+    assert create(16000, 400, 160, 128, 500.0, 100.0, ctypes.byref(h)) == 1     # fmin >= fmax
+    assert create(0, 400, 160, 128, 0.0, 8000.0, ctypes.byref(h)) == 1          # sr <= 0
+    assert create(16000, 400, 160, 128, 0.0, 8000.0, None) == 1                 # null out
+    assert not h.value
+
+
+def test_null_handles_are_rejected(cdll):
+    nf = cdll.logmel_num_frames
+    nf.restype = ctypes.c_int64
+    nf.argtypes = [ctypes.c_void_p, ctypes.c_int64]
+    assert nf(None, 16000) == -1
+    comp = cdll.logmel_compute
+    comp.restype = ctypes.c_int
+    comp.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int64] + [ctypes.c_void_p] * 2
+    assert comp(None, None, None, 0, None, None) == 1
+    cdll.logmel_plan_destroy.argtypes = [ctypes.c_void_p]
+    cdll.logmel_plan_destroy(None)
+    cdll.logmel_stream_destroy.argtypes = [ctypes.c_void_p]
+    cdll.logmel_stream_destroy(None)

@@ -1,0 +1,149 @@
+"""GPU parity of the offline path (logmel_compute through the C ABI) against
+the float64 oracle, on the benchmark workloads and the edge cases."""
+import numpy as np
+import pytest
+
+import oracle as O
+import workloads as W
+from _tolerance import FLOOR32, check_against_oracle
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def plan(lib):
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return lib.Plan()
+
+
+def _run(plan, pcm, off):
+    x = torch.from_numpy(np.ascontiguousarray(pcm, np.float32)).cuda()
+    out = plan.compute(x, off)
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
+def test_three_tone_1s(plan):
+    x = W.three_tone(16000, seed=0)
+    g = _run(plan, x, [0, len(x)])
+    L, M = O.log_mel(x, return_energy=True)
+    assert g.shape == (98, 128)
+    s = check_against_oracle(g, L, M)
+    assert s["zero_cells"] == 98 * 4          # filters 0, 3, 6, 13 hold no bin
+
+
+def test_dense_batch_small_full_compare(plan):
+    pcm, off = W.dense_batch(4)
+    g = _run(plan, pcm, off)
+    L, M = O.log_mel_batch(pcm, off, return_energy=True)
+    check_against_oracle(g, L, M)
+
+
+def test_ragged_batch_small_full_compare(plan):
+    pcm, off = W.ragged_batch(n_utt=24, seed=33)
+    g = _run(plan, pcm, off)
+    L, M = O.log_mel_batch(pcm, off, return_energy=True)
+    check_against_oracle(g, L, M)
+
+
+def _sample_rows(fo, n_random, seed):
+    rng = np.random.default_rng(seed)
+    rows = set(rng.integers(0, fo[-1], n_random).tolist())
+    for u in range(len(fo) - 1):
+        n = fo[u + 1] - fo[u]
+        for t in (0, 1, 31, 32, 33, n - 2, n - 1):
+            if 0 <= t < n:
+                rows.add(int(fo[u] + t))
+    return np.array(sorted(rows), np.int64)
+
+
+def test_dense_batch_full_size_sampled(plan):
+    pcm, off = W.dense_batch(64)
+    g = _run(plan, pcm, off)
+    fo = O.frame_offsets(off)
+    assert g.shape == (64 * 2998, 128)
+    rows = _sample_rows(fo, 1500, 2)
+    L, M = O.log_mel_frames(pcm, off, rows)
+    check_against_oracle(g[rows], L, M)
+
+
+def test_ragged_batch_full_size_sampled(plan):
+    pcm, off = W.ragged_batch()
+    g = _run(plan, pcm, off)
+    fo = O.frame_offsets(off)
+    assert g.shape == (fo[-1], 128)
+    rows = _sample_rows(fo, 1500, 3)
+    L, M = O.log_mel_frames(pcm, off, rows)
+    check_against_oracle(g[rows], L, M)
+
+
+def test_long_form_full_size(plan):
+    pcm, off = W.long_form()
+    g = _run(plan, pcm, off)
+    fo = O.frame_offsets(off)
+    assert g.shape == (174 * 2998, 128) == (521_652, 128)
+    # every all-zero frame must be the exact floor in every band
+    nz = np.concatenate([[0], np.cumsum(pcm != 0, dtype=np.int64)])
+    silent = []
+    for u in range(len(off) - 1):
+        t = np.arange(fo[u + 1] - fo[u])
+        s0 = off[u] + 160 * t
+        silent.append((nz[s0 + 400] - nz[s0]) == 0)
+    silent = np.concatenate(silent)
+    assert silent.sum() > 50_000
+    assert np.all(g[silent] == FLOOR32)
+    rows = _sample_rows(fo, 1500, 4)
+    L, M = O.log_mel_frames(pcm, off, rows)
+    check_against_oracle(g[rows], L, M)
+
+
+def test_edge_lengths_and_unaligned_offsets(plan):
+    lengths = [0, 399, 400, 401, 559, 560, 160 * 31 + 400, 160 * 32 + 400, 160 * 63 + 400, 17, 16000, 3]
+    rng = np.random.default_rng(8)
+    pcm = rng.uniform(-1, 1, 5 + sum(lengths)).astype(np.float32)
+    off = 5 + W.offsets_from_lengths(lengths)           # offsets[0] = 5: odd, unaligned starts
+    g = _run(plan, pcm, off)
+    L, M = O.log_mel_batch(pcm, off, return_energy=True)
+    assert g.shape[0] == O.frame_offsets(off)[-1] == sum(O.num_frames(n) for n in lengths)
+    check_against_oracle(g, L, M)
+
+
+def test_zero_input_is_exact_floor(plan):
+    g = _run(plan, np.zeros(48000, np.float32), [0, 48000])
+    assert g.shape == (298, 128) and np.all(g == FLOOR32)
+
+
+def test_empty_batches(plan):
+    x = torch.zeros(1000, device="cuda")
+    assert plan.compute(x, [0]).shape == (0, 128)
+    assert plan.compute(x, [0, 100, 399, 399]).shape == (0, 128)
+
+
+@pytest.mark.parametrize("n_mels,fmin,fmax", [(80, 20.0, 7600.0), (201, 0.0, 8000.0), (1, 100.0, 4000.0),
+                                              (40, 0.0, 8000.0)])
+def test_other_filterbanks(lib, n_mels, fmin, fmax):
+    p = lib.Plan(n_mels=n_mels, fmin=fmin, fmax=fmax)
+    pcm, off = W.ragged_batch(lengths=[16000, 7000, 30000], seed0=77)
+    g = _run(p, pcm, off)
+    L, M = O.log_mel_batch(pcm, off, O.Params(n_mels=n_mels, fmin=fmin, fmax=fmax), return_energy=True)
+    check_against_oracle(g, L, M)
+
+
+def test_bitwise_deterministic(plan):
+    pcm, off = W.ragged_batch(n_utt=8, seed=12)
+    a = _run(plan, pcm, off)
+    b = _run(plan, pcm, off)
+    assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+
+
+def test_errors_are_reported(lib, plan):
+    x = torch.zeros(1000, device="cuda")
+    with pytest.raises(lib.LogMelError) as e:
+        plan.compute(x, [0, 500, 400])
+    assert e.value.code == 1
+    with pytest.raises(lib.LogMelError) as e:
+        lib.Plan(hop=100)
+    assert e.value.code == 2
+    assert plan.device_status() == 0

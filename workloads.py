@@ -160,10 +160,26 @@ def long_form(total: int = 83_520_000, seed: int = 4, silence_p: float = 0.2, se
     return pcm, offsets_from_lengths(lengths)
 
 
+def _speech_rows(args):
+    n_samples, seeds = args
+    return np.stack([speech_like(n_samples, s) for s in seeds])
+
+
 def stream_signals(n_streams: int = 1024, n_samples: int = 768_000, seed0: int = 5000,
-                   first: int = 0) -> np.ndarray:
-    """Config 5: [n_streams, n_samples] float32, stream s seeded with seed0 + first + s."""
+                   first: int = 0, workers: int = 0) -> np.ndarray:
+    """Config 5: [n_streams, n_samples] float32, stream s seeded with seed0 + first + s.
+    ``workers`` > 1 generates in a spawn-started process pool (same values)."""
     out = np.empty((n_streams, n_samples), np.float32)
+    seeds = [seed0 + first + s for s in range(n_streams)]
+    if workers and workers > 1 and n_streams > 1:
+        import multiprocessing as mp
+        from concurrent.futures import ProcessPoolExecutor
+        step = max(1, n_streams // (4 * workers))
+        jobs = [(n_samples, seeds[i:i + step]) for i in range(0, n_streams, step)]
+        with ProcessPoolExecutor(workers, mp_context=mp.get_context("spawn")) as ex:
+            for i, rows in zip(range(0, n_streams, step), ex.map(_speech_rows, jobs)):
+                out[i:i + rows.shape[0]] = rows
+        return out
     for s in range(n_streams):
-        out[s] = speech_like(n_samples, seed0 + first + s)
+        out[s] = speech_like(n_samples, seeds[s])
     return out
