@@ -75,12 +75,19 @@ int64_t frames_of(int64_t n) { return n < NFFT ? 0 : (n - NFFT) / HOP + 1; }
 
 }  // namespace
 
+struct LaunchCfg {
+  int groups = 0;        // tile groups (of 160 threads) per CTA
+  int group_bytes = 0;   // shared memory per tile group
+  int span_blocks = 0;
+  size_t smem = 0;       // dynamic shared memory per CTA
+  int max_ctas = 0;      // resident CTAs on the device
+};
+
 struct logmel_plan {
   int sr = 0, n_fft = 0, hop = 0, n_mels = 0;
   float fmin = 0.f, fmax = 0.f;
   int device = 0;
-  int max_ctas = 0;
-  size_t smem_bytes = 0;
+  LaunchCfg off{}, str{};    // offline and streaming launch shapes
   Tables* d_tables = nullptr;
   int* d_status = nullptr;
   unsigned char* d_meta = nullptr;
@@ -157,6 +164,14 @@ const char* logmel_status_string(logmel_status s) {
 
 static logmel_status build_tables(Tables* t) {
   std::memset(t, 0, sizeof(Tables));
+  // e^{-2 pi i k / 400} = c - i s, k = 0..399, as (c, c, s, s): the pass-A
+  // twiddle e^{-2 pi i m2 k1 / 200} is entry 2 m2 k1; the real split uses
+  // u_k = -i e^{-2 pi i k / 400}
+  for (int k = 0; k < NFFT; ++k) {
+    double c, s;
+    cos_sin_2pi(k, NFFT, &c, &s);
+    t->w400[k] = make_float4((float)c, (float)c, (float)s, (float)s);
+  }
   // window pairs for pass A: sample n = 20 m1 + 2 m2 and n + 1
   for (int m2 = 0; m2 < N2; ++m2)
     for (int m1 = 0; m1 < N1; ++m1) {
@@ -165,22 +180,6 @@ static logmel_status build_tables(Tables* t) {
       const double w1 = 0.54 - 0.46 * std::cos(2.0 * M_PI * (n + 1) / (NFFT - 1));
       t->win[m2][m1] = make_float2((float)w0, (float)w1);
     }
-  // pass-A twiddles e^{-2 pi i m2 k1 / 200} = c - i s
-  for (int m2 = 0; m2 < N2; ++m2)
-    for (int k1 = 0; k1 < N1; ++k1) {
-      double c, s;
-      cos_sin_2pi((long)m2 * k1, NFFT / 2, &c, &s);
-      t->tw[m2][k1] = make_float4((float)c, (float)c, (float)s, (float)s);
-      t->twn[m2][k1] = make_float2((float)-s, (float)-s);
-    }
-  // real-split twiddles u_k = -i e^{-2 pi i k / 400} = -sin - i cos
-  for (int k = 0; k < NFFT / 2; ++k) {
-    double c, s;
-    cos_sin_2pi(k, NFFT, &c, &s);
-    const double ur = -s, ui = -c;
-    t->post[k] = make_float4((float)ur, (float)ur, (float)ui, (float)ui);
-    t->postn[k] = make_float2((float)-ui, (float)-ui);
-  }
   return LOGMEL_OK;
 }
 
@@ -243,30 +242,47 @@ static logmel_status build_mel(logmel_plan* p) {
   return LOGMEL_OK;
 }
 
+static void shape_launch(LaunchCfg& c, int span_blocks, int n_mels, int max_smem) {
+  c.span_blocks = span_blocks;
+  c.group_bytes = group_bytes_for(span_floats_for(span_blocks, n_mels));
+  c.groups = MAX_TILE_GROUPS;
+  while (c.groups > 1 && TAB_BYTES + (size_t)c.groups * c.group_bytes > (size_t)max_smem) --c.groups;
+  c.smem = TAB_BYTES + (size_t)c.groups * c.group_bytes;
+}
+
 template <bool kDefault>
 static logmel_status setup_kernel(logmel_plan* p, int sms) {
+  const size_t mx = std::max(p->off.smem, p->str.smem);
   if (cudaFuncSetAttribute(logmel_fused_kernel<kDefault>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)p->smem_bytes) != cudaSuccess)
+                           (int)mx) != cudaSuccess)
     return LOGMEL_ERR_CUDA;
-  int occ = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, logmel_fused_kernel<kDefault>, THREADS,
-                                                    p->smem_bytes) != cudaSuccess ||
-      occ < 1)
-    return LOGMEL_ERR_CUDA;
-  p->max_ctas = sms * occ;
+  for (LaunchCfg* c : {&p->off, &p->str}) {
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, logmel_fused_kernel<kDefault>,
+                                                      c->groups * GROUP_THREADS, c->smem) != cudaSuccess ||
+        occ < 1)
+      return LOGMEL_ERR_CUDA;
+    c->max_ctas = sms * occ;
+  }
   return LOGMEL_OK;
 }
 
-static cudaError_t launch(const logmel_plan* p, Args& a, int grid, cudaStream_t s) {
+static cudaError_t launch(const logmel_plan* p, Args& a, int64_t tiles, cudaStream_t s) {
+  const LaunchCfg& c = a.mode == 0 ? p->off : p->str;
+  a.tables = p->d_tables;
+  a.span_blocks = c.span_blocks;
+  a.group_bytes = c.group_bytes;
   std::memcpy(a.mel_w, p->mel.mel_w, sizeof a.mel_w);
   std::memcpy(a.mel_lo, p->mel.mel_lo, sizeof a.mel_lo);
   std::memcpy(a.mel_cnt, p->mel.mel_cnt, sizeof a.mel_cnt);
   std::memcpy(a.mel_woff, p->mel.mel_woff, sizeof a.mel_woff);
   std::memcpy(a.warp_band, p->mel.warp_band, sizeof a.warp_band);
+  const int grid = (int)std::min<int64_t>((tiles + c.groups - 1) / c.groups, c.max_ctas);
+  const int block = c.groups * GROUP_THREADS;
   if (p->default_mel)
-    logmel_fused_kernel<true><<<grid, THREADS, p->smem_bytes, s>>>(a);
+    logmel_fused_kernel<true><<<grid, block, c.smem, s>>>(a);
   else
-    logmel_fused_kernel<false><<<grid, THREADS, p->smem_bytes, s>>>(a);
+    logmel_fused_kernel<false><<<grid, block, c.smem, s>>>(a);
   return cudaGetLastError();
 }
 
@@ -308,7 +324,11 @@ logmel_status logmel_plan_create(int sr, int n_fft, int hop, int n_mels, float f
   int sms = 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, p->device) != cudaSuccess)
     return fail(LOGMEL_ERR_CUDA);
-  p->smem_bytes = sizeof(Smem);
+  int max_smem = 0;
+  if (cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, p->device) != cudaSuccess)
+    return fail(LOGMEL_ERR_CUDA);
+  shape_launch(p->off, OFFLINE_SPAN_BLOCKS, p->n_mels, max_smem);
+  shape_launch(p->str, STREAM_SPAN_BLOCKS, p->n_mels, max_smem);
   st = p->default_mel ? setup_kernel<true>(p, sms) : setup_kernel<false>(p, sms);
   if (st != LOGMEL_OK) return fail(st);
   if (cudaMalloc(&p->d_tables, sizeof(Tables)) != cudaSuccess) return fail(LOGMEL_ERR_OOM);
@@ -440,7 +460,6 @@ logmel_status logmel_compute(logmel_plan* p, const float* pcm, const int64_t* of
   slot.used = true;
   MetaView dv = meta_view(p->d_meta, n_utt);
   Args a{};
-  a.tables = p->d_tables;
   a.out = out;
   a.status = p->d_status;
   a.mode = 0;
@@ -451,8 +470,7 @@ logmel_status logmel_compute(logmel_plan* p, const float* pcm, const int64_t* of
   a.frame_off = dv.frame_off;
   a.tile_off = dv.tile_off;
   a.n_utt = (int)n_utt;
-  const int grid = (int)std::min<int64_t>(tiles, p->max_ctas);
-  CK(launch(p, a, grid, s));
+  CK(launch(p, a, tiles, s));
   return LOGMEL_OK;
 }
 
@@ -522,7 +540,6 @@ static logmel_status push_impl(logmel_stream* st, int base, int count, const flo
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (len > 0) {
     Args a{};
-    a.tables = p->d_tables;
     a.out = out;
     a.status = p->d_status;
     a.mode = 1;
@@ -539,8 +556,7 @@ static logmel_status push_impl(logmel_stream* st, int base, int count, const flo
     a.tps = (int)tps;
     a.update_carry = tps == 1 ? 1 : 0;
     a.out_cap = cap;
-    const int grid = (int)std::min<int64_t>(tiles, p->max_ctas);
-    CK(launch(p, a, grid, s));
+    CK(launch(p, a, tiles, s));
     if (tps > 1) {
       carry_update_kernel<<<count, 128, 0, s>>>(st->d_carry, st->d_carry_len, chunks, chunk_stride,
                                                 len, base);

@@ -47,7 +47,6 @@ constexpr int N2 = 10;
 constexpr int ROLES = 10;             // threads per frame pair in each pass
 constexpr int THREADS = DUOS * ROLES; // 160
 constexpr int BLK = 162;              // smem floats per hop block (160 + 2 pad)
-constexpr int SPAN_BLOCKS = 44;       // >= sum over groups of (frames + 3)
 constexpr int PSTRIDE = NBINS - 2;    // power rows hold bins 1..199 (odd stride: conflict-free)
 constexpr int YROW = N2;              // float4 per pass-A output row
 constexpr int YDUO = N1 * YROW + 1;   // float4 per frame pair (odd: conflict-free by lane = pair)
@@ -63,13 +62,11 @@ constexpr int CARRY_CAP = NFFT;           // carried samples per stream (< 400)
 constexpr float LOG_FLOOR = -23.025850929940457f;
 constexpr float ENERGY_FLOOR = 1e-10f;
 
-// Constant tables, built in float64 on the host by the plan and rounded to fp32.
+// FFT tables, built in float64 on the host by the plan and rounded to fp32;
+// one copy in shared memory serves every tile group of a CTA.
 struct __align__(16) Tables {
+  float4 w400[NFFT];           // (c, c, s, s): e^{-2 pi i k / 400} = c - i s
   float2 win[N2][N1];          // (w[20 m1 + 2 m2], w[20 m1 + 2 m2 + 1]) at [m2][m1]
-  float4 tw[N2][N1];           // (c, c, s, s): e^{-2 pi i m2 k1 / 200} = c - i s
-  float2 twn[N2][N1];          // (-s, -s)
-  float4 post[NFFT / 2];       // (ur, ur, ui, ui): u_k = -i e^{-2 pi i k / 400}
-  float2 postn[NFFT / 2];      // (-ui, -ui)
 };
 
 // One contiguous run of a tile's frames taken from one source signal.
@@ -98,6 +95,8 @@ struct Args {
   int* status;
   int mode;             // 0: offline ragged batch, 1: streaming push
   int num_tiles;
+  int span_blocks;      // hop blocks the span region holds
+  int group_bytes;      // shared memory per tile group
   int n_mels;
   // offline
   const float* pcm;
@@ -220,22 +219,43 @@ __device__ __forceinline__ cx sel(bool p, const cx& a, const cx& b) {
 }
 
 // ---------------------------------------------------------------------------
-// shared memory layout
+// shared memory layout: [tables] then, per tile group of 160 threads,
+// [control block][pass buffer][span region]
+//   pass buffer  pass-A output (float4 per complex pair), then the power rows
+//   span region  staged samples, then the staged output [band][OSTRIDE]
+// A CTA runs several independent tile groups (named barriers per group), so
+// the tables are held once per CTA.  The span region's size is a launch
+// parameter (offline tiles need 34 hop blocks, streaming tiles with four
+// groups 40).
 // ---------------------------------------------------------------------------
-struct __align__(16) Smem {
-  Tables tab;
-  float4 y[DUOS * YDUO];                 // pass A -> pass B; later the staged output
-  float span[SPAN_BLOCKS * BLK];         // staged samples; later the power spectra
+constexpr int GROUP_THREADS = 160;
+constexpr int MAX_TILE_GROUPS = 3;
+struct __align__(16) Ctl {
   Group groups[MAX_GROUPS];
   int64_t slot_row[TILE];
   int slot_block[TILE];
   int ngroups;
   int nslots;
 };
-static_assert(MAX_MELS * OSTRIDE <= DUOS * YDUO * 4, "staged output must fit the pass buffer");
-static_assert(TILE * PSTRIDE <= SPAN_BLOCKS * BLK, "power buffer must fit the span buffer");
+constexpr int TAB_BYTES = (int)((sizeof(Tables) + 127) / 128 * 128);
+constexpr int CTL_BYTES = (int)((sizeof(Ctl) + 127) / 128 * 128);
+constexpr int YBUF_BYTES = DUOS * YDUO * 16;
+constexpr int OFFLINE_SPAN_BLOCKS = 34;   // 32 frames: 31 * 160 + 400 samples
+constexpr int STREAM_SPAN_BLOCKS = 40;    // 4 groups of up to 8 frames
+static_assert(TILE * PSTRIDE * 4 <= YBUF_BYTES, "power rows must fit the pass buffer");
 static_assert(sizeof(mel_default::WARP_BAND) == sizeof(int) * (MEL_WARPS + 1), "default band split must match the mel warps");
-static_assert(sizeof(Tables) % 16 == 0, "tables are copied as float4");
+static_assert(THREADS == GROUP_THREADS, "a tile group is one tile's threads");
+
+__host__ __device__ constexpr int span_floats_for(int span_blocks, int n_mels) {
+  return span_blocks * BLK > n_mels * OSTRIDE ? span_blocks * BLK : n_mels * OSTRIDE;
+}
+__host__ __device__ constexpr int group_bytes_for(int span_floats) {
+  return (CTL_BYTES + YBUF_BYTES + span_floats * 4 + 127) / 128 * 128;
+}
+
+__device__ __forceinline__ void group_sync(int g) {
+  asm volatile("bar.sync %0, %1;" ::"r"(g + 1), "r"(GROUP_THREADS) : "memory");
+}
 
 // Ampere-style asynchronous global -> shared copies (4 or 8 bytes, L1-allocating).
 __device__ __forceinline__ void cp_async4(float* dst, const float* src) {
@@ -258,7 +278,7 @@ __device__ __forceinline__ float src_at(const Group& g, int64_t pos) {
 }
 
 // Thread 0: the tile's groups (sources, frames, span blocks, output rows).
-__device__ void setup_tile(Smem& S, const Args& a, int tile) {
+__device__ void setup_tile(Ctl& S, const Args& a, int tile) {
   int ng = 0, slot = 0, block = 0;
   if (a.mode == 0) {
     int lo = 0, hi = a.n_utt - 1;   // last u with tile_off[u] <= tile
@@ -302,8 +322,9 @@ __device__ void setup_tile(Smem& S, const Args& a, int tile) {
       g.src1 = a.chunks + (int64_t)sl * a.chunk_stride;
       g.len0 = c;
       g.start = f0 * HOP;
-      const int64_t end = min64(B, g.start + (int64_t)HOP * cnt + NFFT);
-      g.nstage = (int)max64(0, end - g.start);
+      // stage the frames' samples; a group with no frames (a push too short
+      // to complete one) stages the whole buffer, which becomes the carry
+      g.nstage = cnt > 0 ? HOP * (cnt - 1) + NFFT : (int)min64(B, NFFT);
       g.nframes = cnt;
       g.slot0 = slot;
       g.block0 = block;
@@ -320,8 +341,8 @@ __device__ void setup_tile(Smem& S, const Args& a, int tile) {
       block += (g.nstage + HOP - 1) / HOP;
     }
   }
-  if (block > SPAN_BLOCKS || slot > TILE) {
-    atomicExch(a.status, block > SPAN_BLOCKS ? STATUS_SPAN_OVERFLOW : STATUS_SLOT_OVERFLOW);
+  if (block > a.span_blocks || slot > TILE) {
+    atomicExch(a.status, block > a.span_blocks ? STATUS_SPAN_OVERFLOW : STATUS_SLOT_OVERFLOW);
     ng = 0;
     slot = 0;
   }
@@ -372,41 +393,51 @@ __device__ __forceinline__ void mel_generic_warp(const Args& a, int w, const flo
 // pass B real split for one pair slot: Z[k] (zk) and Z[200 - k] (zm) ->
 // |2 X[k]|^2 and |2 X[200 - k]|^2 for the two frames of the pair
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void split_power(const Smem& S, const cx& zk, const cx& zm, int k,
+__device__ __forceinline__ void split_power(const Tables& tab, const cx& zk, const cx& zm, int k,
                                             float2& pk, float2& pm) {
   const float2 Ar = add2(zk.re, zm.re), Ai = sub2(zk.im, zm.im);   // A = Z[k] + conj Z[-k]
   const float2 Br = sub2(zk.re, zm.re), Bi = add2(zk.im, zm.im);   // B = Z[k] - conj Z[-k]
-  const float4 u = S.tab.post[k];
-  const float2 nui = S.tab.postn[k];
-  const float2 ur = make_float2(u.x, u.y), ui = make_float2(u.z, u.w);
-  const float2 Tr = fma2(Bi, nui, mul2(Br, ur));                    // T = u_k B
-  const float2 Ti = fma2(Br, ui, mul2(Bi, ur));
-  const float2 pr = add2(Ar, Tr), pi = add2(Ai, Ti);                // 2 X[k]
-  const float2 qr = sub2(Ar, Tr), qi = sub2(Ai, Ti);                // 2 conj X[200 - k]
+  const float4 t = tab.w400[k];                                    // e^{-2 pi i k/400} = c - i s
+  const float2 c = make_float2(t.x, t.y), sn = make_float2(t.z, t.w);
+  // T = u_k B with u_k = -i e^{-2 pi i k / 400} = -s - i c:
+  //   Tr = c Bi - s Br,  Q = -Ti = s Bi + c Br
+  const float2 Tr = sub2(mul2(Bi, c), mul2(Br, sn));
+  const float2 Q = fma2(Bi, sn, mul2(Br, c));
+  const float2 pr = add2(Ar, Tr), pi = sub2(Ai, Q);                 // 2 X[k]
+  const float2 qr = sub2(Ar, Tr), qi = add2(Ai, Q);                 // 2 conj X[200 - k]
   pk = fma2(pi, pi, mul2(pr, pr));
   pm = fma2(qi, qi, mul2(qr, qr));
 }
 
 template <bool kDefaultMel>
-__global__ void __launch_bounds__(THREADS, 2) logmel_fused_kernel(const __grid_constant__ Args a) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  Smem& S = *reinterpret_cast<Smem*>(smem_raw);
-  const int tid = threadIdx.x;
+__global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fused_kernel(const __grid_constant__ Args a) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  const int G = blockDim.x / GROUP_THREADS;
+  const int grp = threadIdx.x / GROUP_THREADS;
+  const int tid = threadIdx.x - grp * GROUP_THREADS;
   const int warp = tid >> 5, lane = tid & 31;
   const int half = lane >> 4, d = lane & 15;       // frame pair d = slots (d, d + 16)
   const int role = 2 * warp + half;               // pass A: m2; pass B: k1 pair index
 
-  {  // constant tables -> shared memory, once per CTA
+  Tables& tab = *reinterpret_cast<Tables*>(smem_raw);
+  {  // FFT tables -> shared memory, once per CTA
     const float4* src = reinterpret_cast<const float4*>(a.tables);
-    float4* dst = reinterpret_cast<float4*>(&S.tab);
-    for (int i = tid; i < (int)(sizeof(Tables) / 16); i += THREADS) dst[i] = src[i];
+    float4* dst = reinterpret_cast<float4*>(smem_raw);
+    for (int i = threadIdx.x; i < (int)(sizeof(Tables) / 16); i += blockDim.x) dst[i] = src[i];
   }
+  __syncthreads();
+  unsigned char* gbase = smem_raw + TAB_BYTES + (size_t)grp * a.group_bytes;
+  Ctl& S = *reinterpret_cast<Ctl*>(gbase);
+  float4* const Y = reinterpret_cast<float4*>(gbase + CTL_BYTES);
+  float* const span = reinterpret_cast<float*>(gbase + CTL_BYTES + YBUF_BYTES);
+  float* const Pbuf = reinterpret_cast<float*>(Y);   // power rows, after pass B has read Y
+  float* const outS = span;                          // staged output, after pass A
 
   const int n_mels = a.n_mels;
-  for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
-    __syncthreads();   // previous tile fully written out; tables visible
+  for (int tile = blockIdx.x * G + grp; tile < a.num_tiles; tile += gridDim.x * G) {
+    group_sync(grp);   // previous tile fully written out
     if (tid == 0) setup_tile(S, a, tile);
-    __syncthreads();
+    group_sync(grp);
     const int ng = S.ngroups;
 
     // ---- stage: each group's span -> hop blocks of BLK floats ---------------
@@ -414,7 +445,7 @@ __global__ void __launch_bounds__(THREADS, 2) logmel_fused_kernel(const __grid_c
     // round trip); 8-byte copies when the source is 8-byte aligned.
     for (int gi = 0; gi < ng; ++gi) {
       const Group& g = S.groups[gi];
-      float* dst = S.span + g.block0 * BLK;
+      float* dst = span + g.block0 * BLK;
       const float* base = g.src0 + g.start;
       if (g.src1 == nullptr && (reinterpret_cast<uintptr_t>(base) & 7) == 0 && (g.nstage & 1) == 0) {
         for (int i = 2 * tid; i < g.nstage; i += 2 * THREADS) {
@@ -444,17 +475,18 @@ __global__ void __launch_bounds__(THREADS, 2) logmel_fused_kernel(const __grid_c
       S.slot_row[tid] = row;
     }
     cp_async_wait_all();
-    __syncthreads();
+    group_sync(grp);
 
     // ---- streaming: write each owned stream's new carry from the span -----
     for (int gi = 0; gi < ng; ++gi) {
       const Group& g = S.groups[gi];
       if (g.carry_len_dst == nullptr) continue;
-      const float* src = S.span + g.block0 * BLK;
+      const float* src = span + g.block0 * BLK;
       for (int i = tid; i < g.new_carry_len; i += THREADS) {
-        const int p = g.carry_from + i;
+        const int p = g.carry_from + i;   // past the staged frames: from the chunk
         const int b = p / HOP;
-        g.carry_dst[i] = src[b * BLK + (p - b * HOP)];
+        g.carry_dst[i] = p < g.nstage ? src[b * BLK + (p - b * HOP)]
+                                      : g.src1[g.start + p - g.len0];
       }
       if (tid == 0) *g.carry_len_dst = g.new_carry_len;
     }
@@ -462,37 +494,36 @@ __global__ void __launch_bounds__(THREADS, 2) logmel_fused_kernel(const __grid_c
     // ---- pass A: window, 20-point DFTs over m1, twiddle --------------------
     {
       const int m2 = role;
-      const float* sa = S.span + BLK * S.slot_block[d] + 2 * m2;
-      const float* sb = S.span + BLK * S.slot_block[d + DUOS] + 2 * m2;
+      const float* sa = span + BLK * S.slot_block[d] + 2 * m2;
+      const float* sb = span + BLK * S.slot_block[d + DUOS] + 2 * m2;
       cx z[N1];
 #pragma unroll
       for (int m1 = 0; m1 < N1; ++m1) {
         const int off = BLK * (m1 / 8) + 20 * (m1 % 8);   // sample n = 20 m1 + 2 m2
         const float2 xa = *reinterpret_cast<const float2*>(sa + off);
         const float2 xb = *reinterpret_cast<const float2*>(sb + off);
-        const float2 w = S.tab.win[m2][m1];
+        const float2 w = tab.win[m2][m1];
         z[m1].re = make_float2(xa.x * w.x, xb.x * w.x);
         z[m1].im = make_float2(xa.y * w.y, xb.y * w.y);
       }
       dft20(z);
-      float4* yrow = S.y + d * YDUO + m2;
+      float4* yrow = Y + d * YDUO + m2;
 #pragma unroll
       for (int k1 = 0; k1 < N1; ++k1) {
         cx v = z[pos20(k1)];
         if (k1 > 0) {
-          const float4 t = S.tab.tw[m2][k1];
-          const float2 ns = S.tab.twn[m2][k1];
+          const float4 t = tab.w400[2 * m2 * k1];   // e^{-2 pi i m2 k1 / 200} = c - i s
           const float2 c = make_float2(t.x, t.y), sn = make_float2(t.z, t.w);
           // (re + i im)(c - i s) = (re c + im s) + i (im c - re s)
           const float2 re = fma2(v.im, sn, mul2(v.re, c));
-          const float2 im = fma2(v.re, ns, mul2(v.im, c));
+          const float2 im = sub2(mul2(v.im, c), mul2(v.re, sn));
           v.re = re;
           v.im = im;
         }
         yrow[k1 * YROW] = make_float4(v.re.x, v.re.y, v.im.x, v.im.y);
       }
     }
-    __syncthreads();
+    group_sync(grp);
 
     // ---- pass B: 10-point DFTs over m2, real split, power -----------------
     {
@@ -500,26 +531,27 @@ __global__ void __launch_bounds__(THREADS, 2) logmel_fused_kernel(const __grid_c
       const bool r0 = (r == 0);
       const int ka = r, kb = r0 ? 10 : N1 - r;
       cx za[N2], zb[N2];
-      const float4* ya = S.y + d * YDUO + ka * YROW;
-      const float4* yb = S.y + d * YDUO + kb * YROW;
+      const float4* ya = Y + d * YDUO + ka * YROW;
+      const float4* yb = Y + d * YDUO + kb * YROW;
 #pragma unroll
       for (int m2 = 0; m2 < N2; ++m2) {
         const float4 va = ya[m2], vb = yb[m2];
         za[m2] = cx{make_float2(va.x, va.y), make_float2(va.z, va.w)};
         zb[m2] = cx{make_float2(vb.x, vb.y), make_float2(vb.z, vb.w)};
       }
+      group_sync(grp);   // every thread holds its rows: the power rows may overwrite Y
       dft10(za);
       dft10(zb);
       // za[pos10(k2)] = Z[ka + 20 k2], zb[pos10(k2)] = Z[kb + 20 k2].
-      float* PA = S.span + d * PSTRIDE - 1;            // frame slot d, bin k at PA[k]
-      float* PB = S.span + (d + DUOS) * PSTRIDE - 1;   // frame slot d + 16
+      float* PA = Pbuf + d * PSTRIDE - 1;            // frame slot d, bin k at PA[k]
+      float* PB = Pbuf + (d + DUOS) * PSTRIDE - 1;   // frame slot d + 16
       if (warp != 0) {
         // roles 2..9: slot j couples Z[k], k = r + 20 j, with Z[200 - k] = zb[9 - j]
 #pragma unroll
         for (int j = 0; j < N2; ++j) {
           const int k = r + 20 * j;
           float2 pk, pm;
-          split_power(S, za[pos10(j)], zb[pos10(9 - j)], k, pk, pm);
+          split_power(tab, za[pos10(j)], zb[pos10(9 - j)], k, pk, pm);
           PA[k] = pk.x;
           PB[k] = pk.y;
           PA[200 - k] = pm.x;
@@ -538,7 +570,7 @@ __global__ void __launch_bounds__(THREADS, 2) logmel_fused_kernel(const __grid_c
                                 : sel(r0, zb[pos10(14 - j)], zb[pos10(9 - j)]);
           const int k = r0 ? (j < 5 ? 20 * j : 10 + 20 * (j - 5)) : r + 20 * j;
           float2 pk, pm;
-          split_power(S, zk, zm, k, pk, pm);
+          split_power(tab, zk, zm, k, pk, pm);
           if (k > 0) {
             PA[k] = pk.x;
             PB[k] = pk.y;
@@ -555,12 +587,12 @@ __global__ void __launch_bounds__(THREADS, 2) logmel_fused_kernel(const __grid_c
         }
       }
     }
-    __syncthreads();
+    group_sync(grp);
 
     // ---- mel + log: warp = band group, lane = frame slot ------------------
     {
-      const float* P = S.span + lane * PSTRIDE - 1;
-      float* o = reinterpret_cast<float*>(S.y);
+      const float* P = Pbuf + lane * PSTRIDE - 1;
+      float* o = outS;
       if constexpr (kDefaultMel) {
         switch (warp) {
           case 0: mel_default_warp<0>(P, o, lane, a.mel_w); break;
@@ -573,11 +605,11 @@ __global__ void __launch_bounds__(THREADS, 2) logmel_fused_kernel(const __grid_c
         mel_generic_warp(a, warp, P, o, lane);
       }
     }
-    __syncthreads();
+    group_sync(grp);
 
     // ---- store: rows of n_mels fp32, one warp per row ---------------------
     {
-      const float* o = reinterpret_cast<const float*>(S.y);
+      const float* o = outS;
       const int ns = S.nslots;
       for (int s = warp; s < ns; s += MEL_WARPS) {
         float* row = a.out + S.slot_row[s] * n_mels;
