@@ -238,6 +238,8 @@ static logmel_status build_mel(logmel_plan* p) {
     same = (mel_default::CNT[i] == a.mel_cnt[i]) && (mel_default::WOFF[i] == a.mel_woff[i]) &&
            (mel_default::CNT[i] == 0 || mel_default::LO[i] == a.mel_lo[i]);
   for (int w = 0; same && w <= MEL_WARPS; ++w) same = mel_default::WARP_BAND[w] == a.warp_band[w];
+  for (int i = 0; same && i < mel_default::NNZ; ++i)   // compiled weights, bit for bit
+    same = std::memcmp(&mel_default::W[i], &a.mel_w[i], sizeof(float)) == 0;
   p->default_mel = same;
   return LOGMEL_OK;
 }

@@ -354,29 +354,44 @@ __device__ void setup_tile(Ctl& S, const Args& a, int tile) {
 // mel stage: lane = frame slot s, P = that frame's power row (bins 1..199 at
 // P[k - 1]), o = staged output [band][OSTRIDE]
 // ---------------------------------------------------------------------------
+// ln(max(M, 1e-10)) with the exact floor constant below 1e-10; above it the
+// hardware base-2 logarithm times ln 2 (M >= 1e-10 is normal, so flushing
+// subnormal inputs changes nothing).
 __device__ __forceinline__ float log_floor(float acc) {
-  return acc < ENERGY_FLOOR ? LOG_FLOOR : __logf(acc);
+  float l2;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(l2) : "f"(acc));
+  return acc < ENERGY_FLOOR ? LOG_FLOOR : l2 * 0.69314718055994531f;
 }
 
 // Default 128-band layout, unrolled at compile time: bins and weight offsets
 // are constants, the weights come from the constant parameter bank.
+// sum_j W[WO + j] * P[LO + j] for j < CNT, in order, weights as immediates
+template <int LO, int WO, int J, int CNT>
+struct MelDot {
+  static __device__ __forceinline__ float run(const float* __restrict__ P, float acc) {
+    if constexpr (J < CNT) {
+      constexpr float w = mel_default::W[WO + J];
+      return MelDot<LO, WO, J + 1, CNT>::run(P, fmaf(w, P[LO + J], acc));
+    } else {
+      return acc;
+    }
+  }
+};
+
 template <int M, int MEND>
 struct MelBands {
-  static __device__ __forceinline__ void run(const float* P, float* o, int s, const float* w) {
+  static __device__ __forceinline__ void run(const float* __restrict__ P, float* __restrict__ o, int s) {
     if constexpr (M < MEND) {
       constexpr int lo = mel_default::LO[M], cnt = mel_default::CNT[M], wo = mel_default::WOFF[M];
-      float acc = 0.f;
-#pragma unroll
-      for (int j = 0; j < cnt; ++j) acc = fmaf(w[wo + j], P[lo + j], acc);
-      o[M * OSTRIDE + s] = log_floor(acc);
-      MelBands<M + 1, MEND>::run(P, o, s, w);
+      o[M * OSTRIDE + s] = log_floor(MelDot<lo, wo, 0, cnt>::run(P, 0.f));
+      MelBands<M + 1, MEND>::run(P, o, s);
     }
   }
 };
 
 template <int W>
-__device__ __forceinline__ void mel_default_warp(const float* P, float* o, int s, const float* w) {
-  MelBands<mel_default::WARP_BAND[W], mel_default::WARP_BAND[W + 1]>::run(P, o, s, w);
+__device__ __forceinline__ void mel_default_warp(const float* __restrict__ P, float* __restrict__ o, int s) {
+  MelBands<mel_default::WARP_BAND[W], mel_default::WARP_BAND[W + 1]>::run(P, o, s);
 }
 
 __device__ __forceinline__ void mel_generic_warp(const Args& a, int w, const float* P, float* o, int s) {
@@ -442,22 +457,30 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
 
     // ---- stage: each group's span -> hop blocks of BLK floats ---------------
     // cp.async puts every load of the span in flight at once (no register
-    // round trip); 8-byte copies when the source is 8-byte aligned.
+    // round trip): 8-byte copies when the source is 8-byte aligned, else
+    // 4-byte; chunk c of a thread lands at a compile-time offset.
     for (int gi = 0; gi < ng; ++gi) {
       const Group& g = S.groups[gi];
       float* dst = span + g.block0 * BLK;
       const float* base = g.src0 + g.start;
-      if (g.src1 == nullptr && (reinterpret_cast<uintptr_t>(base) & 7) == 0 && (g.nstage & 1) == 0) {
-        for (int i = 2 * tid; i < g.nstage; i += 2 * THREADS) {
-          const int b = i / HOP;
-          cp_async8(dst + b * BLK + (i - b * HOP), base + i);
-        }
+      const int n = g.nstage;   // <= 31 * 160 + 400 (frames) or < 400 (carry only)
+      if (g.src1 == nullptr && (reinterpret_cast<uintptr_t>(base) & 7) == 0) {
+        const int hb = (2 * tid) >= HOP;                 // 2 tid + 320 q sits in block 2 q + hb
+        float* d0 = dst + hb * BLK + 2 * tid - hb * HOP;
+        const float* s0 = base + 2 * tid;
+#pragma unroll
+        for (int q = 0; q < (31 * HOP + NFFT + 2 * HOP - 1) / (2 * HOP); ++q)
+          if (2 * tid + 2 * HOP * q < n) cp_async8(d0 + 2 * BLK * q, s0 + 2 * HOP * q);
+      } else if (g.src1 == nullptr) {
+#pragma unroll
+        for (int q = 0; q < (31 * HOP + NFFT + HOP - 1) / HOP; ++q)
+          if (tid + HOP * q < n) cp_async4(dst + BLK * q + tid, base + tid + HOP * q);
       } else {
-        for (int i = tid; i < g.nstage; i += THREADS) {
-          const int64_t pos = g.start + i;
-          const float* src = pos < g.len0 ? g.src0 + pos : g.src1 + (pos - g.len0);
-          const int b = i / HOP;
-          cp_async4(dst + b * BLK + (i - b * HOP), src);
+#pragma unroll 2
+        for (int q = 0; q < (31 * HOP + NFFT + HOP - 1) / HOP; ++q) {
+          const int64_t pos = g.start + tid + HOP * q;
+          if (tid + HOP * q < n)
+            cp_async4(dst + BLK * q + tid, pos < g.len0 ? g.src0 + pos : g.src1 + (pos - g.len0));
         }
       }
     }
@@ -502,7 +525,8 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
         const int off = BLK * (m1 / 8) + 20 * (m1 % 8);   // sample n = 20 m1 + 2 m2
         const float2 xa = *reinterpret_cast<const float2*>(sa + off);
         const float2 xb = *reinterpret_cast<const float2*>(sb + off);
-        const float2 w = tab.win[m2][m1];
+        const float4 w4 = *reinterpret_cast<const float4*>(&tab.win[m2][m1 & ~1]);
+        const float2 w = (m1 & 1) ? make_float2(w4.z, w4.w) : make_float2(w4.x, w4.y);
         z[m1].re = make_float2(xa.x * w.x, xb.x * w.x);
         z[m1].im = make_float2(xa.y * w.y, xb.y * w.y);
       }
@@ -595,11 +619,11 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
       float* o = outS;
       if constexpr (kDefaultMel) {
         switch (warp) {
-          case 0: mel_default_warp<0>(P, o, lane, a.mel_w); break;
-          case 1: mel_default_warp<1>(P, o, lane, a.mel_w); break;
-          case 2: mel_default_warp<2>(P, o, lane, a.mel_w); break;
-          case 3: mel_default_warp<3>(P, o, lane, a.mel_w); break;
-          default: mel_default_warp<4>(P, o, lane, a.mel_w); break;
+          case 0: mel_default_warp<0>(P, o, lane); break;
+          case 1: mel_default_warp<1>(P, o, lane); break;
+          case 2: mel_default_warp<2>(P, o, lane); break;
+          case 3: mel_default_warp<3>(P, o, lane); break;
+          default: mel_default_warp<4>(P, o, lane); break;
         }
       } else {
         mel_generic_warp(a, warp, P, o, lane);
@@ -611,9 +635,23 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
     {
       const float* o = outS;
       const int ns = S.nslots;
-      for (int s = warp; s < ns; s += MEL_WARPS) {
-        float* row = a.out + S.slot_row[s] * n_mels;
-        for (int m = lane; m < n_mels; m += 32) row[m] = o[m * OSTRIDE + s];
+      if constexpr (kDefaultMel) {
+        constexpr int NM = mel_default::N_MELS;
+#pragma unroll
+        for (int r = 0; r < (TILE + MEL_WARPS - 1) / MEL_WARPS; ++r) {
+          const int s = warp + MEL_WARPS * r;
+          if (s < ns) {
+            float* row = a.out + S.slot_row[s] * NM + lane;
+            const float* src = o + lane * OSTRIDE + s;
+#pragma unroll
+            for (int q = 0; q < NM / 32; ++q) row[32 * q] = src[32 * q * OSTRIDE];
+          }
+        }
+      } else {
+        for (int s = warp; s < ns; s += MEL_WARPS) {
+          float* row = a.out + S.slot_row[s] * n_mels;
+          for (int m = lane; m < n_mels; m += 32) row[m] = o[m * OSTRIDE + s];
+        }
       }
     }
   }
