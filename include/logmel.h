@@ -61,6 +61,11 @@ typedef struct logmel_stream logmel_stream;
 /* Human-readable name of a status code (static string, never NULL). */
 const char* logmel_status_string(logmel_status s);
 
+/* The CUDA error behind the last LOGMEL_ERR_CUDA returned on this host
+ * thread: error name, message and the failing call ("" if none).  The
+ * string is thread-local and valid until the next failing call. */
+const char* logmel_last_error(void);
+
 /* Creates a plan on the current CUDA device: builds the Hamming window,
  * FFT twiddles and the mel filterbank in float64 on the host, rounds them
  * to fp32 and uploads them (section 2.3, steps 2-4; preprocessor config

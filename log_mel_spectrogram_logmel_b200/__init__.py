@@ -3,7 +3,7 @@
 Argument marshalling only: every step of the log-mel pipeline runs in the
 CUDA library ``liblogmel_b200.so`` built in this directory.  PyTorch supplies
 device memory and the current CUDA stream.  Importing fails loudly when the
-library has not been built (``python -m log_mel_spectrogram_logmel_b200.build``).
+library has not been built (``python log_mel_spectrogram_logmel_b200/build.py``).
 
     import torch, log_mel_spectrogram_logmel_b200 as lm
     plan = lm.Plan()                                  # sr 16000, n_fft 400, hop 160, 128 mels, 0-8 kHz
@@ -33,7 +33,10 @@ STATUS = {
 class LogMelError(RuntimeError):
     def __init__(self, code: int, what: str):
         self.code = code
-        super().__init__(f"{what}: {STATUS.get(code, code)} ({_lib.logmel_status_string(code).decode()})")
+        msg = f"{what}: {STATUS.get(code, code)} ({_lib.logmel_status_string(code).decode()})"
+        if code == 3:
+            msg += ": " + _lib.logmel_last_error().decode()
+        super().__init__(msg)
 
 
 def lib_path() -> str:
@@ -41,13 +44,14 @@ def lib_path() -> str:
 
 
 if not os.path.exists(_LIB_PATH):
-    raise ImportError(f"{_LIB_PATH} is missing; build it with `python -m log_mel_spectrogram_logmel_b200.build`")
+    raise ImportError(f"{_LIB_PATH} is missing; build it with `python log_mel_spectrogram_logmel_b200/build.py`")
 _lib = ctypes.CDLL(_LIB_PATH)
 
 _p, _i, _i64, _f, _vp = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p
 _i64p = ctypes.POINTER(ctypes.c_int64)
 _SIGS = {
     "logmel_status_string": (ctypes.c_char_p, [_i]),
+    "logmel_last_error": (ctypes.c_char_p, []),
     "logmel_plan_create": (_i, [_i, _i, _i, _i, _f, _f, ctypes.POINTER(_p)]),
     "logmel_plan_destroy": (None, [_p]),
     "logmel_num_frames": (_i64, [_p, _i64]),

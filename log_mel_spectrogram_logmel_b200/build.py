@@ -1,6 +1,8 @@
 """Builds the in-tree CUDA library liblogmel_b200.so for sm_100a with nvcc.
 
-    python -m log_mel_spectrogram_logmel_b200.build
+    python log_mel_spectrogram_logmel_b200/build.py [--force]
+
+(Run it as a script: the package's __init__ loads the library this builds.)
 """
 from __future__ import annotations
 

@@ -10,6 +10,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 #include <new>
 #include <vector>
@@ -78,6 +79,7 @@ int64_t frames_of(int64_t n) { return n < NFFT ? 0 : (n - NFFT) / HOP + 1; }
 struct LaunchCfg {
   int groups = 0;        // tile groups (of 160 threads) per CTA
   int group_bytes = 0;   // shared memory per tile group
+  int ybuf_bytes = 0;    // pass buffer per tile group
   int span_blocks = 0;
   size_t smem = 0;       // dynamic shared memory per CTA
   int max_ctas = 0;      // resident CTAs on the device
@@ -92,6 +94,8 @@ struct logmel_plan {
   int* d_status = nullptr;
   unsigned char* d_meta = nullptr;
   size_t meta_cap = 0;
+  TileDesc* d_tiles = nullptr;    // offline tile descriptors (kernel-written scratch)
+  size_t tiles_cap = 0;
   PinnedSlot ring[RING];
   size_t ring_cap = 0;
   int ring_next = 0;
@@ -141,13 +145,24 @@ __global__ void carry_update_kernel(float* carry, int* carry_len, const float* c
 // ---------------------------------------------------------------------------
 // C ABI
 // ---------------------------------------------------------------------------
-#define CK(call)                                   \
-  do {                                             \
-    cudaError_t e_ = (call);                       \
-    if (e_ != cudaSuccess) return LOGMEL_ERR_CUDA; \
+// Text of the last failed CUDA call on this host thread (logmel_last_error).
+static thread_local char g_last_error[256] = "";
+
+static logmel_status cuda_fail(cudaError_t e, const char* call, int line) {
+  snprintf(g_last_error, sizeof g_last_error, "%s: %s (%s, logmel.cu:%d)", cudaGetErrorName(e),
+           cudaGetErrorString(e), call, line);
+  return LOGMEL_ERR_CUDA;
+}
+
+#define CK(call)                                           \
+  do {                                                     \
+    cudaError_t e_ = (call);                               \
+    if (e_ != cudaSuccess) return cuda_fail(e_, #call, __LINE__); \
   } while (0)
 
 extern "C" {
+
+const char* logmel_last_error(void) { return g_last_error; }
 
 const char* logmel_status_string(logmel_status s) {
   switch (s) {
@@ -246,7 +261,8 @@ static logmel_status build_mel(logmel_plan* p) {
 
 static void shape_launch(LaunchCfg& c, int span_blocks, int n_mels, int max_smem) {
   c.span_blocks = span_blocks;
-  c.group_bytes = group_bytes_for(span_floats_for(span_blocks, n_mels));
+  c.ybuf_bytes = ybuf_bytes_for(n_mels);
+  c.group_bytes = group_bytes_for(span_blocks, n_mels);
   c.groups = MAX_TILE_GROUPS;
   while (c.groups > 1 && TAB_BYTES + (size_t)c.groups * c.group_bytes > (size_t)max_smem) --c.groups;
   c.smem = TAB_BYTES + (size_t)c.groups * c.group_bytes;
@@ -271,9 +287,18 @@ static logmel_status setup_kernel(logmel_plan* p, int sms) {
 
 static cudaError_t launch(const logmel_plan* p, Args& a, int64_t tiles, cudaStream_t s) {
   const LaunchCfg& c = a.mode == 0 ? p->off : p->str;
+  {
+    const cudaError_t pending = cudaGetLastError();
+    if (pending != cudaSuccess) {
+      cuda_fail(pending, "error pending before the launch", __LINE__);
+      return pending;
+    }
+  }
   a.tables = p->d_tables;
   a.span_blocks = c.span_blocks;
   a.group_bytes = c.group_bytes;
+  a.ybuf_bytes = c.ybuf_bytes;
+  a.bulk_store = p->default_mel && (reinterpret_cast<uintptr_t>(a.out) & 15) == 0;
   std::memcpy(a.mel_w, p->mel.mel_w, sizeof a.mel_w);
   std::memcpy(a.mel_lo, p->mel.mel_lo, sizeof a.mel_lo);
   std::memcpy(a.mel_cnt, p->mel.mel_cnt, sizeof a.mel_cnt);
@@ -285,7 +310,14 @@ static cudaError_t launch(const logmel_plan* p, Args& a, int64_t tiles, cudaStre
     logmel_fused_kernel<true><<<grid, block, c.smem, s>>>(a);
   else
     logmel_fused_kernel<false><<<grid, block, c.smem, s>>>(a);
-  return cudaGetLastError();
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    char what[96];
+    snprintf(what, sizeof what, "launch grid %d block %d smem %zu tiles %lld", grid, block, c.smem,
+             (long long)tiles);
+    cuda_fail(e, what, __LINE__);
+  }
+  return e;
 }
 
 extern "C" {
@@ -355,6 +387,7 @@ void logmel_plan_destroy(logmel_plan* p) {
   cudaFree(p->d_tables);
   cudaFree(p->d_status);
   cudaFree(p->d_meta);
+  cudaFree(p->d_tiles);
   for (int i = 0; i < RING; ++i) {
     if (p->ring[i].host) cudaFreeHost(p->ring[i].host);
     if (p->ring[i].done) cudaEventDestroy(p->ring[i].done);
@@ -398,7 +431,7 @@ static logmel_status ensure_meta(logmel_plan* p, size_t bytes) {
   if (bytes > p->ring_cap) {
     for (int i = 0; i < RING; ++i) {
       if (p->ring[i].used) CK(cudaEventSynchronize(p->ring[i].done));
-      if (p->ring[i].host) cudaFreeHost(p->ring[i].host);
+      if (p->ring[i].host) CK(cudaFreeHost(p->ring[i].host));
       p->ring[i].host = nullptr;
       p->ring[i].used = false;
     }
@@ -412,7 +445,7 @@ static logmel_status ensure_meta(logmel_plan* p, size_t bytes) {
   }
   if (bytes > p->meta_cap) {
     CK(cudaDeviceSynchronize());
-    cudaFree(p->d_meta);
+    CK(cudaFree(p->d_meta));
     p->d_meta = nullptr;
     size_t cap = std::max<size_t>(bytes, 4096);
     if (cudaMalloc(&p->d_meta, cap) != cudaSuccess) {
@@ -440,10 +473,21 @@ logmel_status logmel_compute(logmel_plan* p, const float* pcm, const int64_t* of
   }
   if (frames == 0) return LOGMEL_OK;
   if (!pcm || !out) return LOGMEL_ERR_INVALID_ARG;
-  if (tiles >= INT32_MAX) return LOGMEL_ERR_INPUT_TOO_LONG;
+  if (tiles >= INT32_MAX || frames >= INT32_MAX) return LOGMEL_ERR_INPUT_TOO_LONG;
   const size_t bytes = meta_bytes(n_utt);
   st = ensure_meta(p, bytes);
   if (st != LOGMEL_OK) return st;
+  if ((size_t)tiles > p->tiles_cap) {
+    CK(cudaDeviceSynchronize());
+    CK(cudaFree(p->d_tiles));
+    p->d_tiles = nullptr;
+    const size_t cap = std::max<size_t>((size_t)tiles, 1024);
+    if (cudaMalloc(&p->d_tiles, cap * sizeof(TileDesc)) != cudaSuccess) {
+      p->tiles_cap = 0;
+      return LOGMEL_ERR_OOM;
+    }
+    p->tiles_cap = cap;
+  }
   PinnedSlot& slot = p->ring[p->ring_next];
   p->ring_next = (p->ring_next + 1) % RING;
   if (slot.used) CK(cudaEventSynchronize(slot.done));
@@ -465,6 +509,7 @@ logmel_status logmel_compute(logmel_plan* p, const float* pcm, const int64_t* of
   a.out = out;
   a.status = p->d_status;
   a.mode = 0;
+  a.tiles = p->d_tiles;
   a.num_tiles = (int)tiles;
   a.n_mels = p->n_mels;
   a.pcm = pcm;
@@ -472,7 +517,7 @@ logmel_status logmel_compute(logmel_plan* p, const float* pcm, const int64_t* of
   a.frame_off = dv.frame_off;
   a.tile_off = dv.tile_off;
   a.n_utt = (int)n_utt;
-  CK(launch(p, a, tiles, s));
+  if (launch(p, a, tiles, s) != cudaSuccess) return LOGMEL_ERR_CUDA;
   return LOGMEL_OK;
 }
 
@@ -538,7 +583,7 @@ static logmel_status push_impl(logmel_stream* st, int base, int count, const flo
   const int spt = max_n <= TILE / 4 ? 4 : (max_n <= TILE / 2 ? 2 : 1);
   const int64_t tps = max_n <= TILE ? 1 : (max_n + TILE - 1) / TILE;
   const int64_t tiles = (int64_t)((count + spt - 1) / spt) * tps;
-  if (tiles >= INT32_MAX || (int64_t)count * cap >= ((int64_t)1 << 40)) return LOGMEL_ERR_INPUT_TOO_LONG;
+  if (tiles >= INT32_MAX || (int64_t)count * cap >= INT32_MAX) return LOGMEL_ERR_INPUT_TOO_LONG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (len > 0) {
     Args a{};
@@ -558,7 +603,7 @@ static logmel_status push_impl(logmel_stream* st, int base, int count, const flo
     a.tps = (int)tps;
     a.update_carry = tps == 1 ? 1 : 0;
     a.out_cap = cap;
-    CK(launch(p, a, tiles, s));
+    if (launch(p, a, tiles, s) != cudaSuccess) return LOGMEL_ERR_CUDA;
     if (tps > 1) {
       carry_update_kernel<<<count, 128, 0, s>>>(st->d_carry, st->d_carry_len, chunks, chunk_stride,
                                                 len, base);

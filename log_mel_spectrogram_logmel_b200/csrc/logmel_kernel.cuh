@@ -8,8 +8,10 @@
 // Structure (one persistent kernel, 160 threads, tiles of 32 frames; frame
 // slots d and d + 16 form the pair carried by one thread):
 //   stage   each tile's overlapping sample span is copied from HBM once into
-//           shared memory with cp.async, 162 floats per 160-sample hop block
-//           (the 2 pad floats make pass A's reads bank-conflict free)
+//           shared memory by the bulk-copy (TMA) engine, one copy per
+//           160-sample hop block into 164-float slots (cp.async when the
+//           source is not 16-byte aligned); a half-warp reads 8 frame pairs
+//           x 2 roles, which keeps pass A's strided reads conflict-free
 //   pass A  real FFT-400 as a complex FFT-200 of z[m] = x[2m] + i x[2m+1]
 //           (window applied on load), Cooley-Tukey 200 = 20 x 10: ten
 //           20-point DFTs per frame (prime-factor 4 x 5, no inner twiddles),
@@ -23,7 +25,8 @@
 //           (fully unrolled for the default 128-band filterbank, weights read
 //           from the kernel's constant parameter bank)
 //   log     ln via __logf, exact floor constant when the energy is < 1e-10
-//   store   coalesced rows of n_mels fp32
+//   store   rows of n_mels fp32, transposed into dense rows in shared
+//           memory and written by one bulk copy per run of rows
 // Two frames ride in the two lanes of packed f32x2 arithmetic (add/sub/mul/
 // fma .f32x2), so a frame's arithmetic never depends on its partner frame:
 // a frame gives the same bits whichever tile, slot or partner it lands in,
@@ -46,7 +49,7 @@ constexpr int N1 = 20;                // FFT-200 = N1 x N2, m = N2*m1 + m2, k = 
 constexpr int N2 = 10;
 constexpr int ROLES = 10;             // threads per frame pair in each pass
 constexpr int THREADS = DUOS * ROLES; // 160
-constexpr int BLK = 162;              // smem floats per hop block (160 + 2 pad)
+constexpr int BLK = 164;              // smem floats per hop block: 16-byte aligned (bulk copies)
 constexpr int PSTRIDE = NBINS - 2;    // power rows hold bins 1..199 (odd stride: conflict-free)
 constexpr int YROW = N2;              // float4 per pass-A output row
 constexpr int YDUO = N1 * YROW + 1;   // float4 per frame pair (odd: conflict-free by lane = pair)
@@ -89,14 +92,24 @@ struct Group {
   int carry_from;     // span-relative position of the new carry's first sample
 };
 
+// Offline tile: one run of up to 32 frames of one utterance.
+struct TileDesc {
+  int64_t src;        // sample index of the tile's first frame
+  int out_row;        // output row of the tile's first frame
+  int nframes;
+};
+
 struct Args {
   const Tables* tables;
+  TileDesc* tiles;      // offline: per-tile descriptors (written by the kernel's prologue)
   float* out;
   int* status;
   int mode;             // 0: offline ragged batch, 1: streaming push
   int num_tiles;
   int span_blocks;      // hop blocks the span region holds
   int group_bytes;      // shared memory per tile group
+  int ybuf_bytes;       // pass buffer bytes per tile group
+  int bulk_store;       // 1: rows leave through bulk copies (default layout, aligned out)
   int n_mels;
   // offline
   const float* pcm;
@@ -125,7 +138,7 @@ struct Args {
   short warp_band[MEL_WARPS + 1];
 };
 
-enum DeviceStatus : int { STATUS_OK = 0, STATUS_SPAN_OVERFLOW = 1, STATUS_SLOT_OVERFLOW = 2 };
+enum DeviceStatus : int { STATUS_OK = 0, STATUS_SPAN_OVERFLOW = 1, STATUS_SLOT_OVERFLOW = 2, STATUS_COPY_TIMEOUT = 3 };
 
 // ---------------------------------------------------------------------------
 // packed fp32 pair arithmetic (sm_100a .f32x2): lane x = frame A, lane y = frame B
@@ -220,37 +233,44 @@ __device__ __forceinline__ cx sel(bool p, const cx& a, const cx& b) {
 
 // ---------------------------------------------------------------------------
 // shared memory layout: [tables] then, per tile group of 160 threads,
-// [control block][pass buffer][span region]
-//   pass buffer  pass-A output (float4 per complex pair), then the power rows
-//   span region  staged samples, then the staged output [band][OSTRIDE]
+// [control block x 2][pass buffer][span region]
+//   control      groups and per-slot rows of the current and the next tile
+//   pass buffer  pass-A output (float4 per complex pair); after pass B has
+//                read it, the power rows [32][199] and the staged output
+//                [n_mels][OSTRIDE]
+//   span region  staged samples (the next tile's span is fetched while the
+//                current tile finishes pass B, mel and store)
 // A CTA runs several independent tile groups (named barriers per group), so
-// the tables are held once per CTA.  The span region's size is a launch
-// parameter (offline tiles need 34 hop blocks, streaming tiles with four
-// groups 40).
+// the tables are held once per CTA.  Offline tiles need 34 hop blocks of
+// span, streaming tiles with four groups 40.
 // ---------------------------------------------------------------------------
 constexpr int GROUP_THREADS = 160;
 constexpr int MAX_TILE_GROUPS = 3;
 struct __align__(16) Ctl {
   Group groups[MAX_GROUPS];
-  int64_t slot_row[TILE];
-  int slot_block[TILE];
+  unsigned long long bar;   // mbarrier completing this buffer's bulk span copies
   int ngroups;
   int nslots;
+  int tma;                  // 1: the span arrives by bulk copies (wait on bar)
+  int bar_parity;           // phase of bar to wait for
+  int copy_ok;              // thread 0's verdict on the bulk copies (0: timed out)
+  int pad_;
 };
 constexpr int TAB_BYTES = (int)((sizeof(Tables) + 127) / 128 * 128);
-constexpr int CTL_BYTES = (int)((sizeof(Ctl) + 127) / 128 * 128);
+constexpr int CTL_BYTES = (int)((sizeof(Ctl) + 15) / 16 * 16);
 constexpr int YBUF_BYTES = DUOS * YDUO * 16;
+constexpr int PROWS_FLOATS = TILE * PSTRIDE;
 constexpr int OFFLINE_SPAN_BLOCKS = 34;   // 32 frames: 31 * 160 + 400 samples
 constexpr int STREAM_SPAN_BLOCKS = 40;    // 4 groups of up to 8 frames
-static_assert(TILE * PSTRIDE * 4 <= YBUF_BYTES, "power rows must fit the pass buffer");
 static_assert(sizeof(mel_default::WARP_BAND) == sizeof(int) * (MEL_WARPS + 1), "default band split must match the mel warps");
 static_assert(THREADS == GROUP_THREADS, "a tile group is one tile's threads");
 
-__host__ __device__ constexpr int span_floats_for(int span_blocks, int n_mels) {
-  return span_blocks * BLK > n_mels * OSTRIDE ? span_blocks * BLK : n_mels * OSTRIDE;
+__host__ __device__ constexpr int ybuf_bytes_for(int n_mels) {
+  return (PROWS_FLOATS + n_mels * OSTRIDE) * 4 > YBUF_BYTES ? ((PROWS_FLOATS + n_mels * OSTRIDE) * 4 + 15) / 16 * 16
+                                                           : YBUF_BYTES;
 }
-__host__ __device__ constexpr int group_bytes_for(int span_floats) {
-  return (CTL_BYTES + YBUF_BYTES + span_floats * 4 + 127) / 128 * 128;
+__host__ __device__ constexpr int group_bytes_for(int span_blocks, int n_mels) {
+  return (2 * CTL_BYTES + ybuf_bytes_for(n_mels) + span_blocks * BLK * 4 + 127) / 128 * 128;
 }
 
 __device__ __forceinline__ void group_sync(int g) {
@@ -270,6 +290,47 @@ __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
 }
 
+// --- bulk-copy (TMA) engine and mbarrier helpers --------------------------
+__device__ __forceinline__ unsigned smem_addr(const void* p) {
+  return static_cast<unsigned>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(unsigned long long* bar) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;\n" ::"r"(smem_addr(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(unsigned long long* bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_addr(bar)), "r"(bytes)
+               : "memory");
+}
+// Polls phase `parity` of the barrier (each poll suspends for at most about
+// a microsecond); returns false if it has not completed after `polls` polls.
+__device__ __forceinline__ bool mbar_wait(unsigned long long* bar, int parity, int polls) {
+  const unsigned a = smem_addr(bar);
+  for (int it = 0; it < polls; ++it) {
+    unsigned done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(a), "r"(parity), "r"(1000)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, unsigned bytes, unsigned long long* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                   smem_addr(dst)),
+               "l"(src), "r"(bytes), "r"(smem_addr(bar))
+               : "memory");
+}
+__device__ __forceinline__ void bulk_store(void* dst, const void* src, unsigned bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n" ::"l"(dst), "r"(smem_addr(src)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+
 __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
 __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
 
@@ -277,69 +338,96 @@ __device__ __forceinline__ float src_at(const Group& g, int64_t pos) {
   return pos < g.len0 ? g.src0[pos] : g.src1[pos - g.len0];
 }
 
-// Thread 0: the tile's groups (sources, frames, span blocks, output rows).
-__device__ void setup_tile(Ctl& S, const Args& a, int tile) {
+// Span hop block of frame slot t (slots past the tile's frames read block 0:
+// valid samples whose results are dropped) and its output row (-1: unused).
+__device__ __forceinline__ int slot_block(const Ctl& S, int t) {
+  int b = 0;
+  for (int gi = 0; gi < S.ngroups; ++gi) {
+    const Group& g = S.groups[gi];
+    if (t >= g.slot0 && t < g.slot0 + g.nframes) b = g.block0 + (t - g.slot0);
+  }
+  return b;
+}
+__device__ __forceinline__ int64_t slot_row(const Ctl& S, int t) {
+  int64_t r = -1;
+  for (int gi = 0; gi < S.ngroups; ++gi) {
+    const Group& g = S.groups[gi];
+    if (t >= g.slot0 && t < g.slot0 + g.nframes) r = g.out_row + (t - g.slot0);
+  }
+  return r;
+}
+
+// Offline tile descriptor: binary search of the tile's utterance.
+__device__ TileDesc offline_desc(const Args& a, int tile) {
+  int lo = 0, hi = a.n_utt - 1;   // last u with tile_off[u] <= tile
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (a.tile_off[mid] <= tile) lo = mid; else hi = mid - 1;
+  }
+  const int u = lo;
+  const int64_t f0 = (int64_t)(tile - a.tile_off[u]) * TILE;
+  const int64_t nfr = a.frame_off[u + 1] - a.frame_off[u];
+  TileDesc t;
+  t.src = a.sample_off[u] + f0 * HOP;
+  t.out_row = (int)(a.frame_off[u] + f0);
+  t.nframes = (int)min64(TILE, nfr - f0);
+  return t;
+}
+
+__device__ void setup_offline(Ctl& S, const Args& a, const TileDesc& t) {
+  Group& g = S.groups[0];
+  g.src0 = a.pcm + t.src;
+  g.src1 = nullptr;
+  g.start = 0;
+  g.nframes = t.nframes;
+  g.nstage = HOP * (t.nframes - 1) + NFFT;
+  g.len0 = g.nstage;
+  g.out_row = t.out_row;
+  g.slot0 = 0;
+  g.block0 = 0;
+  g.carry_len_dst = nullptr;
+  S.ngroups = 1;
+  S.nslots = t.nframes;
+  S.tma = (reinterpret_cast<uintptr_t>(g.src0) & 15) == 0;
+}
+
+// Streaming tile (thread 0): up to `spt` streams, each a group of its frames.
+__device__ void setup_stream(Ctl& S, const Args& a, int tile) {
   int ng = 0, slot = 0, block = 0;
-  if (a.mode == 0) {
-    int lo = 0, hi = a.n_utt - 1;   // last u with tile_off[u] <= tile
-    while (lo < hi) {
-      int mid = (lo + hi + 1) >> 1;
-      if (a.tile_off[mid] <= tile) lo = mid; else hi = mid - 1;
-    }
-    const int u = lo;
-    const int64_t f0 = (int64_t)(tile - a.tile_off[u]) * TILE;
-    const int64_t nfr = a.frame_off[u + 1] - a.frame_off[u];
-    const int cnt = (int)min64(TILE, nfr - f0);
-    Group& g = S.groups[0];
-    g.src0 = a.pcm + a.sample_off[u];
-    g.src1 = nullptr;
-    g.len0 = a.sample_off[u + 1] - a.sample_off[u];
+  const int sg = tile / a.tps, st = tile - sg * a.tps;
+  for (int j = 0; j < a.spt; ++j) {
+    const int sl = sg * a.spt + j;
+    if (sl >= a.n_push_streams) break;
+    const int s = a.stream_base + sl;
+    const int c = a.carry_len[s];
+    const int64_t B = c + a.push_len;
+    const int64_t n = B >= NFFT ? (B - NFFT) / HOP + 1 : 0;
+    const int64_t f0 = (int64_t)st * TILE;
+    const int cnt = (int)max64(0, min64(TILE / a.spt, n - f0));
+    const bool owner = (st == 0) && a.update_carry;
+    if (cnt == 0 && !owner) continue;
+    Group& g = S.groups[ng];
+    g.src0 = a.carry + (int64_t)s * CARRY_CAP;
+    g.src1 = a.chunks + (int64_t)sl * a.chunk_stride;
+    g.len0 = c;
     g.start = f0 * HOP;
-    g.out_row = a.frame_off[u] + f0;
+    // stage the frames' samples; a group with no frames (a push too short
+    // to complete one) stages the whole buffer, which becomes the carry
+    g.nstage = cnt > 0 ? HOP * (cnt - 1) + NFFT : (int)min64(B, NFFT);
     g.nframes = cnt;
-    g.nstage = cnt > 0 ? HOP * (cnt - 1) + NFFT : 0;
-    g.slot0 = 0;
-    g.block0 = 0;
+    g.slot0 = slot;
+    g.block0 = block;
+    g.out_row = (int64_t)sl * a.out_cap + f0;
     g.carry_len_dst = nullptr;
-    ng = 1;
-    slot = cnt;
-    block = (g.nstage + HOP - 1) / HOP;
-  } else {
-    const int sg = tile / a.tps, st = tile - sg * a.tps;
-    for (int j = 0; j < a.spt; ++j) {
-      const int sl = sg * a.spt + j;
-      if (sl >= a.n_push_streams) break;
-      const int s = a.stream_base + sl;
-      const int c = a.carry_len[s];
-      const int64_t B = c + a.push_len;
-      const int64_t n = B >= NFFT ? (B - NFFT) / HOP + 1 : 0;
-      const int64_t f0 = (int64_t)st * TILE;
-      const int cnt = (int)max64(0, min64(TILE / a.spt, n - f0));
-      const bool owner = (st == 0) && a.update_carry;
-      if (cnt == 0 && !owner) continue;
-      Group& g = S.groups[ng];
-      g.src0 = a.carry + (int64_t)s * CARRY_CAP;
-      g.src1 = a.chunks + (int64_t)sl * a.chunk_stride;
-      g.len0 = c;
-      g.start = f0 * HOP;
-      // stage the frames' samples; a group with no frames (a push too short
-      // to complete one) stages the whole buffer, which becomes the carry
-      g.nstage = cnt > 0 ? HOP * (cnt - 1) + NFFT : (int)min64(B, NFFT);
-      g.nframes = cnt;
-      g.slot0 = slot;
-      g.block0 = block;
-      g.out_row = (int64_t)sl * a.out_cap + f0;
-      g.carry_len_dst = nullptr;
-      if (owner) {
-        g.carry_dst = a.carry + (int64_t)s * CARRY_CAP;
-        g.carry_len_dst = a.carry_len + s;
-        g.new_carry_len = (int)(B - n * HOP);
-        g.carry_from = (int)(n * HOP - g.start);
-      }
-      ++ng;
-      slot += cnt;
-      block += (g.nstage + HOP - 1) / HOP;
+    if (owner) {
+      g.carry_dst = a.carry + (int64_t)s * CARRY_CAP;
+      g.carry_len_dst = a.carry_len + s;
+      g.new_carry_len = (int)(B - n * HOP);
+      g.carry_from = (int)(n * HOP - g.start);
     }
+    ++ng;
+    slot += cnt;
+    block += (g.nstage + HOP - 1) / HOP;
   }
   if (block > a.span_blocks || slot > TILE) {
     atomicExch(a.status, block > a.span_blocks ? STATUS_SPAN_OVERFLOW : STATUS_SLOT_OVERFLOW);
@@ -348,6 +436,51 @@ __device__ void setup_tile(Ctl& S, const Args& a, int tile) {
   }
   S.ngroups = ng;
   S.nslots = slot;
+  S.tma = 0;
+}
+
+// Issue the cp.async copies of a tile's spans (all threads of the group);
+// chunk q of a thread lands at a compile-time offset.
+__device__ __forceinline__ void stage_tile(Ctl& S, float* span, int tid) {
+  if (S.tma) {   // one bulk copy per hop block (640 B; the last one 320 B), warp 0 issues
+    const Group& g = S.groups[0];
+    if (tid < 32) {
+      const int nb = (g.nstage + HOP - 1) / HOP;
+      if (tid == 0) mbar_expect_tx(&S.bar, (unsigned)g.nstage * 4u);
+      __syncwarp();
+      for (int b = tid; b < nb; b += 32) {
+        const int len = min(HOP, g.nstage - b * HOP);
+        bulk_load(span + (g.block0 + b) * BLK, g.src0 + b * HOP, (unsigned)len * 4u, &S.bar);
+      }
+    }
+    return;
+  }
+  for (int gi = 0; gi < S.ngroups; ++gi) {
+    const Group& g = S.groups[gi];
+    float* dst = span + g.block0 * BLK;
+    const float* base = g.src0 + g.start;
+    const int n = g.nstage;   // <= 31 * 160 + 400 (frames) or < 400 (carry only)
+    if (g.src1 == nullptr && (reinterpret_cast<uintptr_t>(base) & 7) == 0) {
+      const int hb = (2 * tid) >= HOP;                 // 2 tid + 320 q sits in block 2 q + hb
+      float* d0 = dst + hb * BLK + 2 * tid - hb * HOP;
+      const float* s0 = base + 2 * tid;
+#pragma unroll
+      for (int q = 0; q < (31 * HOP + NFFT + 2 * HOP - 1) / (2 * HOP); ++q)
+        if (2 * tid + 2 * HOP * q < n) cp_async8(d0 + 2 * BLK * q, s0 + 2 * HOP * q);
+    } else if (g.src1 == nullptr) {
+#pragma unroll
+      for (int q = 0; q < (31 * HOP + NFFT + HOP - 1) / HOP; ++q)
+        if (tid + HOP * q < n) cp_async4(dst + BLK * q + tid, base + tid + HOP * q);
+    } else {
+#pragma unroll 2
+      for (int q = 0; q < (31 * HOP + NFFT + HOP - 1) / HOP; ++q) {
+        const int64_t pos = g.start + tid + HOP * q;
+        if (tid + HOP * q < n)
+          cp_async4(dst + BLK * q + tid, pos < g.len0 ? g.src0 + pos : g.src1 + (pos - g.len0));
+      }
+    }
+  }
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -365,33 +498,54 @@ __device__ __forceinline__ float log_floor(float acc) {
 
 // Default 128-band layout, unrolled at compile time: bins and weight offsets
 // are constants, the weights come from the constant parameter bank.
-// sum_j W[WO + j] * P[LO + j] for j < CNT, in order, weights as immediates
-template <int LO, int WO, int J, int CNT>
+// sum_j W[WO + j] * p[LO + j - KLO] for j < CNT, in order, weights as
+// immediates, p = the warp's bins held in registers
+template <int KLO, int LO, int WO, int J, int CNT, int NP>
 struct MelDot {
-  static __device__ __forceinline__ float run(const float* __restrict__ P, float acc) {
+  static __device__ __forceinline__ float run(const float (&p)[NP], float acc) {
     if constexpr (J < CNT) {
       constexpr float w = mel_default::W[WO + J];
-      return MelDot<LO, WO, J + 1, CNT>::run(P, fmaf(w, P[LO + J], acc));
+      return MelDot<KLO, LO, WO, J + 1, CNT, NP>::run(p, fmaf(w, p[LO + J - KLO], acc));
     } else {
       return acc;
     }
   }
 };
 
-template <int M, int MEND>
+template <int KLO, int M, int MEND, int NP>
 struct MelBands {
-  static __device__ __forceinline__ void run(const float* __restrict__ P, float* __restrict__ o, int s) {
+  static __device__ __forceinline__ void run(const float (&p)[NP], float* __restrict__ o, int s) {
     if constexpr (M < MEND) {
       constexpr int lo = mel_default::LO[M], cnt = mel_default::CNT[M], wo = mel_default::WOFF[M];
-      o[M * OSTRIDE + s] = log_floor(MelDot<lo, wo, 0, cnt>::run(P, 0.f));
-      MelBands<M + 1, MEND>::run(P, o, s);
+      o[M * OSTRIDE + s] = log_floor(MelDot<KLO, lo, wo, 0, cnt, NP>::run(p, 0.f));
+      MelBands<KLO, M + 1, MEND, NP>::run(p, o, s);
     }
   }
 };
 
+// bins [lo, hi] touched by bands [b0, b1) of the default layout
+__host__ __device__ constexpr int mel_bin_lo(int b0, int b1) {
+  int k = NBINS;
+  for (int m = b0; m < b1; ++m)
+    if (mel_default::CNT[m] > 0 && mel_default::LO[m] < k) k = mel_default::LO[m];
+  return k;
+}
+__host__ __device__ constexpr int mel_bin_hi(int b0, int b1) {
+  int k = 0;
+  for (int m = b0; m < b1; ++m)
+    if (mel_default::CNT[m] > 0 && mel_default::LO[m] + mel_default::CNT[m] - 1 > k)
+      k = mel_default::LO[m] + mel_default::CNT[m] - 1;
+  return k;
+}
+
 template <int W>
 __device__ __forceinline__ void mel_default_warp(const float* __restrict__ P, float* __restrict__ o, int s) {
-  MelBands<mel_default::WARP_BAND[W], mel_default::WARP_BAND[W + 1]>::run(P, o, s);
+  constexpr int B0 = mel_default::WARP_BAND[W], B1 = mel_default::WARP_BAND[W + 1];
+  constexpr int KLO = mel_bin_lo(B0, B1), KHI = mel_bin_hi(B0, B1), NP = KHI - KLO + 1;
+  float p[NP];
+#pragma unroll
+  for (int i = 0; i < NP; ++i) p[i] = P[KLO + i];   // each bin read once
+  MelBands<KLO, B0, B1, NP>::run(p, o, s);
 }
 
 __device__ __forceinline__ void mel_generic_warp(const Args& a, int w, const float* P, float* o, int s) {
@@ -431,8 +585,11 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
   const int grp = threadIdx.x / GROUP_THREADS;
   const int tid = threadIdx.x - grp * GROUP_THREADS;
   const int warp = tid >> 5, lane = tid & 31;
-  const int half = lane >> 4, d = lane & 15;       // frame pair d = slots (d, d + 16)
-  const int role = 2 * warp + half;               // pass A: m2; pass B: k1 pair index
+  // lane -> frame pair d (slots d and d + 16) and role: a half-warp holds 8
+  // pairs x 2 adjacent roles, so its strided span reads hit distinct banks
+  const int d = ((lane >> 4) << 3) | (lane & 7);
+  const int role = 2 * warp + ((lane >> 3) & 1);   // pass A: m2; pass B: k1 pair index
+  const int stride = gridDim.x * G;               // a group's tiles: first + k * stride
 
   Tables& tab = *reinterpret_cast<Tables*>(smem_raw);
   {  // FFT tables -> shared memory, once per CTA
@@ -440,68 +597,65 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
     float4* dst = reinterpret_cast<float4*>(smem_raw);
     for (int i = threadIdx.x; i < (int)(sizeof(Tables) / 16); i += blockDim.x) dst[i] = src[i];
   }
+  if (a.mode == 0) {  // offline: this CTA's tile descriptors, searched in parallel
+    const int rounds = (a.num_tiles + stride - 1) / stride;
+    for (int j = threadIdx.x; j < rounds * G; j += blockDim.x) {
+      const int t = blockIdx.x * G + (j % G) + (j / G) * stride;
+      if (t < a.num_tiles) a.tiles[t] = offline_desc(a, t);
+    }
+  }
   __syncthreads();
+
   unsigned char* gbase = smem_raw + TAB_BYTES + (size_t)grp * a.group_bytes;
-  Ctl& S = *reinterpret_cast<Ctl*>(gbase);
-  float4* const Y = reinterpret_cast<float4*>(gbase + CTL_BYTES);
-  float* const span = reinterpret_cast<float*>(gbase + CTL_BYTES + YBUF_BYTES);
+  Ctl* const ctl0 = reinterpret_cast<Ctl*>(gbase);
+  Ctl* const ctl1 = reinterpret_cast<Ctl*>(gbase + CTL_BYTES);
+  if (tid == 0) {
+    mbar_init(&ctl0->bar);
+    mbar_init(&ctl1->bar);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  int armed0 = 0, armed1 = 0;   // thread 0: bulk-copy uses of each control buffer
+  __syncthreads();
+  float4* const Y = reinterpret_cast<float4*>(gbase + 2 * CTL_BYTES);
+  float* const span = reinterpret_cast<float*>(gbase + 2 * CTL_BYTES + a.ybuf_bytes);
   float* const Pbuf = reinterpret_cast<float*>(Y);   // power rows, after pass B has read Y
-  float* const outS = span;                          // staged output, after pass A
+  float* const outS = Pbuf + PROWS_FLOATS;           // staged output, after the power rows
 
   const int n_mels = a.n_mels;
-  for (int tile = blockIdx.x * G + grp; tile < a.num_tiles; tile += gridDim.x * G) {
-    group_sync(grp);   // previous tile fully written out
-    if (tid == 0) setup_tile(S, a, tile);
+  int tile = blockIdx.x * G + grp;
+  if (tile < a.num_tiles) {
+    if (tid == 0) {
+      if (a.mode == 0) setup_offline(*ctl0, a, a.tiles[tile]);
+      else setup_stream(*ctl0, a, tile);
+      if (ctl0->tma) ctl0->bar_parity = (armed0++) & 1;
+    }
     group_sync(grp);
+    stage_tile(*ctl0, span, tid);
+  }
+  int cur = 0;
+  for (; tile < a.num_tiles; tile += stride, cur ^= 1) {
+    Ctl& S = cur ? *ctl1 : *ctl0;
+    Ctl& N = cur ? *ctl0 : *ctl1;
+    const int next = tile + stride;
+    TileDesc nd;
+    if (tid == 0 && a.mode == 0 && next < a.num_tiles) nd = a.tiles[next];   // used after pass A
+    if (tid == 0) {
+      // thread 0 alone waits for the bulk copies (bounded: ~65 ms), and
+      // publishes the verdict so the whole group takes the same path
+      S.copy_ok = S.tma ? mbar_wait(&S.bar, S.bar_parity, 1 << 16) : 1;
+      bulk_wait_read();   // the previous tile's bulk row copies have read smem
+    }
+    asm volatile("cp.async.wait_all;\n" ::: "memory");
+    group_sync(grp);   // this tile's span is staged; the previous tile's rows are stored
+    if (!S.copy_ok) {   // a bulk copy never completed: flag it and stop this group
+      if (tid == 0) atomicExch(a.status, STATUS_COPY_TIMEOUT);
+      break;
+    }
+    if (S.tma) mbar_wait(&S.bar, S.bar_parity, 1 << 16);   // completed: acquires the copied span
     const int ng = S.ngroups;
 
-    // ---- stage: each group's span -> hop blocks of BLK floats ---------------
-    // cp.async puts every load of the span in flight at once (no register
-    // round trip): 8-byte copies when the source is 8-byte aligned, else
-    // 4-byte; chunk c of a thread lands at a compile-time offset.
-    for (int gi = 0; gi < ng; ++gi) {
-      const Group& g = S.groups[gi];
-      float* dst = span + g.block0 * BLK;
-      const float* base = g.src0 + g.start;
-      const int n = g.nstage;   // <= 31 * 160 + 400 (frames) or < 400 (carry only)
-      if (g.src1 == nullptr && (reinterpret_cast<uintptr_t>(base) & 7) == 0) {
-        const int hb = (2 * tid) >= HOP;                 // 2 tid + 320 q sits in block 2 q + hb
-        float* d0 = dst + hb * BLK + 2 * tid - hb * HOP;
-        const float* s0 = base + 2 * tid;
-#pragma unroll
-        for (int q = 0; q < (31 * HOP + NFFT + 2 * HOP - 1) / (2 * HOP); ++q)
-          if (2 * tid + 2 * HOP * q < n) cp_async8(d0 + 2 * BLK * q, s0 + 2 * HOP * q);
-      } else if (g.src1 == nullptr) {
-#pragma unroll
-        for (int q = 0; q < (31 * HOP + NFFT + HOP - 1) / HOP; ++q)
-          if (tid + HOP * q < n) cp_async4(dst + BLK * q + tid, base + tid + HOP * q);
-      } else {
-#pragma unroll 2
-        for (int q = 0; q < (31 * HOP + NFFT + HOP - 1) / HOP; ++q) {
-          const int64_t pos = g.start + tid + HOP * q;
-          if (tid + HOP * q < n)
-            cp_async4(dst + BLK * q + tid, pos < g.len0 ? g.src0 + pos : g.src1 + (pos - g.len0));
-        }
-      }
-    }
-    if (tid < TILE) {  // per-slot span block and output row
-      int blk = 0;
-      int64_t row = -1;
-      for (int gi = 0; gi < ng; ++gi) {
-        const Group& g = S.groups[gi];
-        if (tid >= g.slot0 && tid < g.slot0 + g.nframes) {
-          blk = g.block0 + (tid - g.slot0);
-          row = g.out_row + (tid - g.slot0);
-        }
-      }
-      S.slot_block[tid] = blk;
-      S.slot_row[tid] = row;
-    }
-    cp_async_wait_all();
-    group_sync(grp);
-
     // ---- streaming: write each owned stream's new carry from the span -----
-    for (int gi = 0; gi < ng; ++gi) {
+    for (int gi = 0; a.mode == 1 && gi < ng; ++gi) {
       const Group& g = S.groups[gi];
       if (g.carry_len_dst == nullptr) continue;
       const float* src = span + g.block0 * BLK;
@@ -517,8 +671,8 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
     // ---- pass A: window, 20-point DFTs over m1, twiddle --------------------
     {
       const int m2 = role;
-      const float* sa = span + BLK * S.slot_block[d] + 2 * m2;
-      const float* sb = span + BLK * S.slot_block[d + DUOS] + 2 * m2;
+      const float* sa = span + BLK * slot_block(S, d) + 2 * m2;
+      const float* sb = span + BLK * slot_block(S, d + DUOS) + 2 * m2;
       cx z[N1];
 #pragma unroll
       for (int m1 = 0; m1 < N1; ++m1) {
@@ -547,6 +701,11 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
         yrow[k1 * YROW] = make_float4(v.re.x, v.re.y, v.im.x, v.im.y);
       }
     }
+    if (tid == 0 && next < a.num_tiles) {   // the next tile's groups
+      if (a.mode == 0) setup_offline(N, a, nd);
+      else setup_stream(N, a, next);
+      if (N.tma) N.bar_parity = cur ? (armed0++) & 1 : (armed1++) & 1;
+    }
     group_sync(grp);
 
     // ---- pass B: 10-point DFTs over m2, real split, power -----------------
@@ -563,7 +722,9 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
         za[m2] = cx{make_float2(va.x, va.y), make_float2(va.z, va.w)};
         zb[m2] = cx{make_float2(vb.x, vb.y), make_float2(vb.z, vb.w)};
       }
-      group_sync(grp);   // every thread holds its rows: the power rows may overwrite Y
+      fence_async_smem();  // this thread's span reads precede the bulk copies into it
+      group_sync(grp);   // rows held in registers: power rows may overwrite Y; span is free
+      if (next < a.num_tiles) stage_tile(N, span, tid);   // fetch the next tile meanwhile
       dft10(za);
       dft10(zb);
       // za[pos10(k2)] = Z[ka + 20 k2], zb[pos10(k2)] = Z[kb + 20 k2].
@@ -616,17 +777,16 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
     // ---- mel + log: warp = band group, lane = frame slot ------------------
     {
       const float* P = Pbuf + lane * PSTRIDE - 1;
-      float* o = outS;
       if constexpr (kDefaultMel) {
         switch (warp) {
-          case 0: mel_default_warp<0>(P, o, lane); break;
-          case 1: mel_default_warp<1>(P, o, lane); break;
-          case 2: mel_default_warp<2>(P, o, lane); break;
-          case 3: mel_default_warp<3>(P, o, lane); break;
-          default: mel_default_warp<4>(P, o, lane); break;
+          case 0: mel_default_warp<0>(P, outS, lane); break;
+          case 1: mel_default_warp<1>(P, outS, lane); break;
+          case 2: mel_default_warp<2>(P, outS, lane); break;
+          case 3: mel_default_warp<3>(P, outS, lane); break;
+          default: mel_default_warp<4>(P, outS, lane); break;
         }
       } else {
-        mel_generic_warp(a, warp, P, o, lane);
+        mel_generic_warp(a, warp, P, outS, lane);
       }
     }
     group_sync(grp);
@@ -637,24 +797,50 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
       const int ns = S.nslots;
       if constexpr (kDefaultMel) {
         constexpr int NM = mel_default::N_MELS;
+        if (a.bulk_store) {
+          // transpose into dense rows (in the dead power-row region), then one
+          // bulk copy per group of consecutive rows
+          float* dense = Pbuf;
 #pragma unroll
-        for (int r = 0; r < (TILE + MEL_WARPS - 1) / MEL_WARPS; ++r) {
-          const int s = warp + MEL_WARPS * r;
-          if (s < ns) {
-            float* row = a.out + S.slot_row[s] * NM + lane;
-            const float* src = o + lane * OSTRIDE + s;
+          for (int rr = 0; rr < (TILE + MEL_WARPS - 1) / MEL_WARPS; ++rr) {
+            const int s = warp + MEL_WARPS * rr;
+            if (s < ns) {
+              const float* src = o + lane * OSTRIDE + s;
 #pragma unroll
-            for (int q = 0; q < NM / 32; ++q) row[32 * q] = src[32 * q * OSTRIDE];
+              for (int q = 0; q < NM / 32; ++q) dense[s * NM + lane + 32 * q] = src[32 * q * OSTRIDE];
+            }
+          }
+          fence_async_smem();
+          group_sync(grp);
+          if (tid == 0) {
+            for (int gi = 0; gi < S.ngroups; ++gi) {
+              const Group& g = S.groups[gi];
+              if (g.nframes > 0)
+                bulk_store(a.out + g.out_row * NM, dense + g.slot0 * NM, (unsigned)g.nframes * NM * 4u);
+            }
+            bulk_commit();
+          }
+        } else {
+#pragma unroll
+          for (int rr = 0; rr < (TILE + MEL_WARPS - 1) / MEL_WARPS; ++rr) {
+            const int s = warp + MEL_WARPS * rr;
+            if (s < ns) {
+              float* row = a.out + slot_row(S, s) * NM + lane;
+              const float* src = o + lane * OSTRIDE + s;
+#pragma unroll
+              for (int q = 0; q < NM / 32; ++q) row[32 * q] = src[32 * q * OSTRIDE];
+            }
           }
         }
       } else {
         for (int s = warp; s < ns; s += MEL_WARPS) {
-          float* row = a.out + S.slot_row[s] * n_mels;
+          float* row = a.out + slot_row(S, s) * n_mels;
           for (int m = lane; m < n_mels; m += 32) row[m] = o[m * OSTRIDE + s];
         }
       }
     }
   }
+  if (tid == 0) asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");   // rows written before exit
 }
 
 }  // namespace logmel

@@ -18,8 +18,8 @@ def _declared():
 
 @pytest.fixture(scope="module")
 def cdll():
-    from log_mel_spectrogram_logmel_b200 import build
-    path = build.build()
+    import __graft_entry__
+    path = __graft_entry__._builder().build()
     return ctypes.CDLL(path)
 
 
