@@ -5,6 +5,8 @@
 // built in float64 and rounded to fp32), the ragged-batch index map (frame
 // and tile prefix sums), the streaming carry state and its checkpoint blob.
 // Device side: logmel_kernel.cuh.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -74,6 +76,22 @@ double mel_to_hz(double m) { return 700.0 * (std::pow(10.0, m / 2595.0) - 1.0); 
 
 int64_t frames_of(int64_t n) { return n < NFFT ? 0 : (n - NFFT) / HOP + 1; }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    cudaGetLastError();
+  }
+  return fn;
+}
+
 }  // namespace
 
 struct LaunchCfg {
@@ -101,6 +119,11 @@ struct logmel_plan {
   int ring_next = 0;
   Args mel{};               // filterbank fields copied into every launch
   bool default_mel = false; // structure equals the compiled default layout
+  // tensor map of the last offline PCM buffer (re-encoded when it changes)
+  CUtensorMap tmap{};
+  const float* tmap_pcm = nullptr;
+  int64_t tmap_len = -1;
+  int tmap_rows = 0;
 };
 
 struct logmel_stream {
@@ -510,6 +533,29 @@ logmel_status logmel_compute(logmel_plan* p, const float* pcm, const int64_t* of
   a.status = p->d_status;
   a.mode = 0;
   a.tiles = p->d_tiles;
+  // the PCM as rows of 160 samples for one-box tile copies (16-byte aligned
+  // base and at least one full row); the box is 164 x 34: columns 160..163
+  // are outside the tensor and arrive as zeros
+  const int64_t total = off[n_utt];
+  if (pcm != p->tmap_pcm || total != p->tmap_len) {
+    p->tmap_pcm = pcm;
+    p->tmap_len = total;
+    p->tmap_rows = 0;
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    const int64_t rows = total / HOP;
+    if (enc && (reinterpret_cast<uintptr_t>(pcm) & 15) == 0 && rows >= 1 && rows < INT32_MAX) {
+      cuuint64_t dims[2] = {(cuuint64_t)HOP, (cuuint64_t)rows};
+      cuuint64_t strides[1] = {(cuuint64_t)HOP * sizeof(float)};
+      cuuint32_t box[2] = {(cuuint32_t)BLK, (cuuint32_t)OFFLINE_SPAN_BLOCKS};
+      cuuint32_t estr[2] = {1, 1};
+      if (enc(&p->tmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(pcm), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+        p->tmap_rows = (int)rows;
+    }
+  }
+  a.tmap = p->tmap;
+  a.tmap_rows = p->tmap_rows;
   a.num_tiles = (int)tiles;
   a.n_mels = p->n_mels;
   a.pcm = pcm;

@@ -33,6 +33,7 @@
 // which is what makes streaming output equal offline output bit for bit.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -100,6 +101,12 @@ struct TileDesc {
 };
 
 struct Args {
+  // offline: the PCM as a 2-D tensor of 160-sample rows; a 164 x 34 box
+  // lands one tile's span in its hop-block slots (columns 160..163 of a box
+  // row are outside the tensor and read as zeros: padding)
+  CUtensorMap tmap;
+  int tmap_rows;        // rows of the tensor (0: no tensor map)
+  int pad_tm_[3];
   const Tables* tables;
   TileDesc* tiles;      // offline: per-tile descriptors (written by the kernel's prologue)
   float* out;
@@ -251,13 +258,13 @@ struct __align__(16) Ctl {
   unsigned long long bar;   // mbarrier completing this buffer's bulk span copies
   int ngroups;
   int nslots;
-  int tma;                  // 1: the span arrives by bulk copies (wait on bar)
+  int tma;                  // 1: per-block bulk copies, 2: one tensor copy (wait on bar)
   int bar_parity;           // phase of bar to wait for
-  int copy_ok;              // thread 0's verdict on the bulk copies (0: timed out)
-  int pad_;
+  int copy_ok;              // the waiting thread's verdict on the bulk copies (0: timed out)
+  int tmap_row;             // tensor row of the span's first sample (tma == 2)
 };
 constexpr int TAB_BYTES = (int)((sizeof(Tables) + 127) / 128 * 128);
-constexpr int CTL_BYTES = (int)((sizeof(Ctl) + 15) / 16 * 16);
+constexpr int CTL_BYTES = (int)((sizeof(Ctl) + 127) / 128 * 128);   // span region 128-byte aligned
 constexpr int YBUF_BYTES = DUOS * YDUO * 16;
 constexpr int PROWS_FLOATS = TILE * PSTRIDE;
 constexpr int OFFLINE_SPAN_BLOCKS = 34;   // 32 frames: 31 * 160 + 400 samples
@@ -265,10 +272,13 @@ constexpr int STREAM_SPAN_BLOCKS = 40;    // 4 groups of up to 8 frames
 static_assert(sizeof(mel_default::WARP_BAND) == sizeof(int) * (MEL_WARPS + 1), "default band split must match the mel warps");
 static_assert(THREADS == GROUP_THREADS, "a tile group is one tile's threads");
 
+// Every region starts on a 128-byte boundary: a tensor bulk copy's shared
+// memory destination must be 128-byte aligned.
 __host__ __device__ constexpr int ybuf_bytes_for(int n_mels) {
-  return (PROWS_FLOATS + n_mels * OSTRIDE) * 4 > YBUF_BYTES ? ((PROWS_FLOATS + n_mels * OSTRIDE) * 4 + 15) / 16 * 16
-                                                           : YBUF_BYTES;
+  return (((PROWS_FLOATS + n_mels * OSTRIDE) * 4 > YBUF_BYTES ? (PROWS_FLOATS + n_mels * OSTRIDE) * 4 : YBUF_BYTES) +
+          127) / 128 * 128;
 }
+static_assert(YBUF_BYTES % 128 == 0 && CTL_BYTES % 128 == 0 && TAB_BYTES % 128 == 0, "128-byte aligned regions");
 __host__ __device__ constexpr int group_bytes_for(int span_blocks, int n_mels) {
   return (2 * CTL_BYTES + ybuf_bytes_for(n_mels) + span_blocks * BLK * 4 + 127) / 128 * 128;
 }
@@ -322,6 +332,14 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, unsigned b
                "l"(src), "r"(bytes), "r"(smem_addr(bar))
                : "memory");
 }
+__device__ __forceinline__ void tensor_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                               unsigned long long* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];\n" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
 __device__ __forceinline__ void bulk_store(void* dst, const void* src, unsigned bytes) {
   asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n" ::"l"(dst), "r"(smem_addr(src)),
                "r"(bytes)
@@ -374,7 +392,7 @@ __device__ TileDesc offline_desc(const Args& a, int tile) {
   return t;
 }
 
-__device__ void setup_offline(Ctl& S, const Args& a, const TileDesc& t) {
+__device__ void setup_offline(Ctl& S, const Args& a, const TileDesc& t, const float* span) {
   Group& g = S.groups[0];
   g.src0 = a.pcm + t.src;
   g.src1 = nullptr;
@@ -388,7 +406,17 @@ __device__ void setup_offline(Ctl& S, const Args& a, const TileDesc& t) {
   g.carry_len_dst = nullptr;
   S.ngroups = 1;
   S.nslots = t.nframes;
-  S.tma = (reinterpret_cast<uintptr_t>(g.src0) & 15) == 0;
+  // one tensor copy when the span starts on a tensor row and its last hop
+  // block is a whole row of the tensor; else per-block bulk copies when the
+  // source is 16-byte aligned; else cp.async
+  const int64_t row = t.src / HOP;
+  const int nb = (g.nstage + HOP - 1) / HOP;
+  if (a.tmap_rows > 0 && t.src % HOP == 0 && row + nb <= a.tmap_rows && (smem_addr(span) & 127) == 0) {
+    S.tma = 2;
+    S.tmap_row = (int)row;
+  } else {
+    S.tma = (reinterpret_cast<uintptr_t>(g.src0) & 15) == 0;
+  }
 }
 
 // Streaming tile (thread 0): up to `spt` streams, each a group of its frames.
@@ -441,14 +469,26 @@ __device__ void setup_stream(Ctl& S, const Args& a, int tile) {
 
 // Issue the cp.async copies of a tile's spans (all threads of the group);
 // chunk q of a thread lands at a compile-time offset.
-__device__ __forceinline__ void stage_tile(Ctl& S, float* span, int tid) {
-  if (S.tma) {   // one bulk copy per hop block (640 B; the last one 320 B), warp 0 issues
+// The thread that arms, issues and first waits on the bulk copies (warp 4,
+// whose pass-B share is the lightest).
+constexpr int COPY_TID = 128;
+
+__device__ __forceinline__ void stage_tile(Ctl& S, float* span, int tid, const Args& a) {
+  if (S.tma == 2) {   // one 164 x 34 tensor box per tile
+    if (tid == COPY_TID) {
+      mbar_expect_tx(&S.bar, (unsigned)(BLK * OFFLINE_SPAN_BLOCKS * 4));
+      tensor_load_2d(span, &a.tmap, 0, S.tmap_row, &S.bar);
+    }
+    return;
+  }
+  if (S.tma) {   // one bulk copy per hop block (640 B; the last one 320 B)
     const Group& g = S.groups[0];
-    if (tid < 32) {
+    if (tid >= COPY_TID && tid < COPY_TID + 32) {
+      const int l = tid - COPY_TID;
       const int nb = (g.nstage + HOP - 1) / HOP;
-      if (tid == 0) mbar_expect_tx(&S.bar, (unsigned)g.nstage * 4u);
+      if (l == 0) mbar_expect_tx(&S.bar, (unsigned)g.nstage * 4u);
       __syncwarp();
-      for (int b = tid; b < nb; b += 32) {
+      for (int b = l; b < nb; b += 32) {
         const int len = min(HOP, g.nstage - b * HOP);
         bulk_load(span + (g.block0 + b) * BLK, g.src0 + b * HOP, (unsigned)len * 4u, &S.bar);
       }
@@ -609,12 +649,12 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
   unsigned char* gbase = smem_raw + TAB_BYTES + (size_t)grp * a.group_bytes;
   Ctl* const ctl0 = reinterpret_cast<Ctl*>(gbase);
   Ctl* const ctl1 = reinterpret_cast<Ctl*>(gbase + CTL_BYTES);
-  if (tid == 0) {
+  if (tid == COPY_TID) {
     mbar_init(&ctl0->bar);
     mbar_init(&ctl1->bar);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
-  int armed0 = 0, armed1 = 0;   // thread 0: bulk-copy uses of each control buffer
+  int armed0 = 0, armed1 = 0;   // COPY_TID: bulk-copy uses of each control buffer
   __syncthreads();
   float4* const Y = reinterpret_cast<float4*>(gbase + 2 * CTL_BYTES);
   float* const span = reinterpret_cast<float*>(gbase + 2 * CTL_BYTES + a.ybuf_bytes);
@@ -624,13 +664,13 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
   const int n_mels = a.n_mels;
   int tile = blockIdx.x * G + grp;
   if (tile < a.num_tiles) {
-    if (tid == 0) {
-      if (a.mode == 0) setup_offline(*ctl0, a, a.tiles[tile]);
+    if (tid == COPY_TID) {
+      if (a.mode == 0) setup_offline(*ctl0, a, a.tiles[tile], span);
       else setup_stream(*ctl0, a, tile);
       if (ctl0->tma) ctl0->bar_parity = (armed0++) & 1;
     }
     group_sync(grp);
-    stage_tile(*ctl0, span, tid);
+    stage_tile(*ctl0, span, tid, a);
   }
   int cur = 0;
   for (; tile < a.num_tiles; tile += stride, cur ^= 1) {
@@ -638,17 +678,17 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
     Ctl& N = cur ? *ctl0 : *ctl1;
     const int next = tile + stride;
     TileDesc nd;
-    if (tid == 0 && a.mode == 0 && next < a.num_tiles) nd = a.tiles[next];   // used after pass A
-    if (tid == 0) {
-      // thread 0 alone waits for the bulk copies (bounded: ~65 ms), and
-      // publishes the verdict so the whole group takes the same path
+    if (tid == COPY_TID && a.mode == 0 && next < a.num_tiles) nd = a.tiles[next];   // used after pass A
+    if (tid == COPY_TID) {
+      // one thread waits for the bulk copies (bounded: ~65 ms), and publishes
+      // the verdict so the whole group takes the same path
       S.copy_ok = S.tma ? mbar_wait(&S.bar, S.bar_parity, 1 << 16) : 1;
-      bulk_wait_read();   // the previous tile's bulk row copies have read smem
     }
+    if (tid == 0) bulk_wait_read();   // the previous tile's bulk row copies have read smem
     asm volatile("cp.async.wait_all;\n" ::: "memory");
     group_sync(grp);   // this tile's span is staged; the previous tile's rows are stored
     if (!S.copy_ok) {   // a bulk copy never completed: flag it and stop this group
-      if (tid == 0) atomicExch(a.status, STATUS_COPY_TIMEOUT);
+      if (tid == COPY_TID) atomicExch(a.status, STATUS_COPY_TIMEOUT);
       break;
     }
     if (S.tma) mbar_wait(&S.bar, S.bar_parity, 1 << 16);   // completed: acquires the copied span
@@ -701,8 +741,8 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
         yrow[k1 * YROW] = make_float4(v.re.x, v.re.y, v.im.x, v.im.y);
       }
     }
-    if (tid == 0 && next < a.num_tiles) {   // the next tile's groups
-      if (a.mode == 0) setup_offline(N, a, nd);
+    if (tid == COPY_TID && next < a.num_tiles) {   // the next tile's groups
+      if (a.mode == 0) setup_offline(N, a, nd, span);
       else setup_stream(N, a, next);
       if (N.tma) N.bar_parity = cur ? (armed0++) & 1 : (armed1++) & 1;
     }
@@ -724,7 +764,7 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
       }
       fence_async_smem();  // this thread's span reads precede the bulk copies into it
       group_sync(grp);   // rows held in registers: power rows may overwrite Y; span is free
-      if (next < a.num_tiles) stage_tile(N, span, tid);   // fetch the next tile meanwhile
+      if (next < a.num_tiles) stage_tile(N, span, tid, a);   // fetch the next tile meanwhile
       dft10(za);
       dft10(zb);
       // za[pos10(k2)] = Z[ka + 20 k2], zb[pos10(k2)] = Z[kb + 20 k2].
