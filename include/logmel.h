@@ -52,7 +52,8 @@ typedef enum {
   LOGMEL_ERR_CUDA = 3,           /* a CUDA runtime call failed               */
   LOGMEL_ERR_OOM = 4,            /* device or pinned allocation failed       */
   LOGMEL_ERR_INPUT_TOO_LONG = 5, /* a count exceeds the kernels' index range */
-  LOGMEL_ERR_DEVICE_STATUS = 6   /* a kernel flagged an inconsistency        */
+  LOGMEL_ERR_DEVICE_STATUS = 6,  /* a kernel flagged an inconsistency        */
+  LOGMEL_ERR_NOALLOC_LIMIT = 7   /* batch beyond logmel_compute_noalloc's fixed scratch */
 } logmel_status;
 
 typedef struct logmel_plan logmel_plan;
@@ -155,6 +156,51 @@ logmel_status logmel_stream_set_state(logmel_stream* st, const void* host_blob, 
 
 /* Empties one stream (or all streams if stream_id < 0), enqueued on `stream`. */
 logmel_status logmel_stream_reset(logmel_stream* st, int stream_id, void* stream);
+
+/* Offline ragged batch that allocates nothing.  (The paper has no
+ * counterpart: this is a deployment variant of logmel_compute.)
+ *
+ * Who needs it: callers that cannot call cudaMalloc -- a process whose
+ * device memory belongs to another allocator (a serving runtime or host
+ * application that reserves the GPU's memory at start-up and hands out
+ * buffers, so a raw cudaMalloc fails or escapes its accounting), and
+ * real-time audio code for which cudaMalloc / cudaFree would block the
+ * thread or synchronise the device.  Creating a plan allocates, so this
+ * entry point takes none: it computes the default front-end (sr 16000,
+ * n_fft 400, hop 160, 128 mels over 0-8000 Hz), the configuration
+ * logmel_plan_create(16000, 400, 160, 128, 0, 8000) describes, with the same
+ * kernel, and its output equals that plan's logmel_compute output.
+ *
+ * Arguments as logmel_compute, without the plan:
+ *   pcm, offsets, n_utt, out   as logmel_compute (out holds sum over u of
+ *                  floor((len_u - 400) / 160) + 1 rows of 128 floats, 0 rows
+ *                  for len_u < 400)
+ *   device_status  device, one int, or NULL: set to 0 on `stream` before the
+ *                  kernel, which stores a nonzero code there if it flags an
+ *                  inconsistency (NULL: a word inside the scratch, unread)
+ * All of pcm, out and device_status must be memory of the current device.
+ *
+ * Scratch and limits: the FFT tables, the status word, the ragged metadata
+ * and the tile descriptors live in one fixed array in device memory (about
+ * 600 KB, held by every GPU that loads this library until the process
+ * exits).  A call takes at most 4096 utterances and 32768 tiles, where
+ * utterance u needs ceil(frames_u / 32) tiles (for example 4096 utterances
+ * of up to 2.5 s, 64 of 30 s, or one of up to 2.9 h); beyond either limit it
+ * returns LOGMEL_ERR_NOALLOC_LIMIT and enqueues nothing.
+ *
+ * Calls and set-up: the first call on each device does a one-time set-up
+ * with that device current -- it looks up the scratch address, uploads the
+ * tables with a synchronous copy and sets the kernel's shared-memory limit
+ * -- so make that first call before any stream capture begins.  Every call
+ * on a device shares the one scratch array, which keeps the last call's
+ * contents: calls whose work overlaps on the GPU (two streams, or two host
+ * threads without ordering) race on it and may return wrong output; order
+ * them on one stream or with events.  Host-side, calls are serialised by a
+ * lock.  Each call copies its metadata host->device from a static host
+ * buffer with cudaMemcpyAsync and launches one kernel; no device or pinned
+ * memory is allocated or freed. */
+logmel_status logmel_compute_noalloc(const float* pcm, const int64_t* offsets, int64_t n_utt,
+                                     float* out, int* device_status, void* stream);
 
 /* Reads and clears the plan's device status word (synchronises `stream`).
  * *code = 0 when no kernel has flagged an inconsistency since the last read. */

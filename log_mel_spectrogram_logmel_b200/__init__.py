@@ -19,7 +19,7 @@ import os
 
 import numpy as np
 
-__all__ = ["Plan", "Stream", "LogMelError", "lib_path", "exported_symbols", "STATUS"]
+__all__ = ["Plan", "Stream", "LogMelError", "compute_noalloc", "lib_path", "exported_symbols", "STATUS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "liblogmel_b200.so")
@@ -27,6 +27,7 @@ _LIB_PATH = os.path.join(_HERE, "liblogmel_b200.so")
 STATUS = {
     0: "LOGMEL_OK", 1: "LOGMEL_ERR_INVALID_ARG", 2: "LOGMEL_ERR_UNSUPPORTED", 3: "LOGMEL_ERR_CUDA",
     4: "LOGMEL_ERR_OOM", 5: "LOGMEL_ERR_INPUT_TOO_LONG", 6: "LOGMEL_ERR_DEVICE_STATUS",
+    7: "LOGMEL_ERR_NOALLOC_LIMIT",
 }
 
 
@@ -58,6 +59,7 @@ _SIGS = {
     "logmel_frame_offsets": (_i, [_p, _i64p, _i64, _i64p]),
     "logmel_total_frames": (_i64, [_p, _i64p, _i64]),
     "logmel_compute": (_i, [_p, _vp, _i64p, _i64, _vp, _vp]),
+    "logmel_compute_noalloc": (_i, [_vp, _i64p, _i64, _vp, _vp, _vp]),
     "logmel_stream_create": (_i, [_p, _i, ctypes.POINTER(_p)]),
     "logmel_stream_destroy": (None, [_p]),
     "logmel_stream_frames_for_push": (_i64, [_p, _i, _i64]),
@@ -116,6 +118,43 @@ def _check_cuda_f32(t, name, device):
         raise ValueError(f"{name} is on {t.device}, the plan on {device}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+
+
+def compute_noalloc(pcm, offsets, out, device_status=None, stream=None):
+    """The allocation-free entry point (logmel_compute_noalloc): the default
+    front-end (sr 16000, n_fft 400, hop 160, 128 mels, 0-8 kHz) of a ragged
+    batch, written into the caller's ``out`` with no device or pinned
+    allocation, for callers whose device memory belongs to another allocator
+    or whose thread must not block in cudaMalloc / cudaFree.
+
+    ``out`` (CUDA float32, at least total_frames x 128) and the optional
+    ``device_status`` (CUDA int32, one element) are the caller's.  At most
+    4096 utterances and 32768 tiles of 32 frames per call; calls that overlap
+    on the GPU share one scratch array and race.  Returns ``out``."""
+    torch = _torch()
+    device = pcm.device if isinstance(pcm, torch.Tensor) else None
+    _check_cuda_f32(pcm, "pcm", device)
+    _check_cuda_f32(out, "out", device)
+    off = _offsets(offsets)
+    if off[-1] > pcm.numel():
+        raise ValueError("offsets reach beyond pcm")
+    n = np.diff(off)
+    if np.any(n < 0) or off[0] < 0:
+        raise ValueError("offsets must be non-negative and non-decreasing")
+    total = int(np.where(n >= 400, (n - 400) // 160 + 1, 0).sum())
+    if out.numel() < total * 128:
+        raise ValueError("out is too small")
+    st = _vp(0)
+    if device_status is not None:
+        if (not isinstance(device_status, torch.Tensor) or device_status.dtype != torch.int32
+                or device_status.device != device or device_status.numel() < 1):
+            raise TypeError("device_status must be an int32 tensor on the device of pcm")
+        st = _vp(device_status.data_ptr())
+    with torch.cuda.device(device):
+        _check(_lib.logmel_compute_noalloc(_vp(pcm.data_ptr()), _ptr64(off), off.shape[0] - 1,
+                                           _vp(out.data_ptr()), st, _stream_handle(stream, device)),
+               "logmel_compute_noalloc")
+    return out
 
 
 class Plan:

@@ -14,6 +14,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -196,6 +197,9 @@ const char* logmel_status_string(logmel_status s) {
     case LOGMEL_ERR_OOM: return "out of memory";
     case LOGMEL_ERR_INPUT_TOO_LONG: return "input too long for the kernels' index range";
     case LOGMEL_ERR_DEVICE_STATUS: return "a kernel flagged an inconsistency";
+    case LOGMEL_ERR_NOALLOC_LIMIT:
+      return "batch larger than the fixed scratch of logmel_compute_noalloc "
+             "(at most 4096 utterances and 32768 tiles of 32 frames)";
   }
   return "unknown status";
 }
@@ -774,3 +778,163 @@ logmel_status logmel_plan_device_status(logmel_plan* p, int* code, void* stream)
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free offline entry point: logmel_compute_noalloc
+//
+// For callers that cannot call cudaMalloc: a process whose device memory is
+// owned by another allocator (a serving runtime or a host application that
+// reserves the GPU's memory at start-up and hands out buffers, so a raw
+// cudaMalloc fails or escapes its accounting), and a real-time audio path on
+// which cudaMalloc / cudaFree would block the host thread or synchronise the
+// device.  The caller still owns pcm and out; everything else the offline
+// kernel needs lives in one fixed array in device memory.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int64_t NOALLOC_MAX_UTT = 4096;     // utterances per call
+constexpr int64_t NOALLOC_MAX_TILES = 32768;  // 32-frame tiles per call (1,048,576 frames)
+constexpr int NOALLOC_MAX_DEVICES = 64;
+
+// Scratch layout: FFT tables | status word | ragged metadata | tile descriptors.
+constexpr size_t NA_TABLES_OFF = 0;
+constexpr size_t NA_STATUS_OFF = (sizeof(Tables) + 255) / 256 * 256;
+constexpr size_t NA_META_OFF = NA_STATUS_OFF + 256;
+constexpr size_t NA_META_CAP =   // meta_bytes(NOALLOC_MAX_UTT), rounded up to 256
+    (16 * (NOALLOC_MAX_UTT + 1) + ((4 * (NOALLOC_MAX_UTT + 1) + 15) & ~15) + 255) / 256 * 256;
+constexpr size_t NA_TILES_OFF = NA_META_OFF + NA_META_CAP;
+constexpr size_t NA_SCRATCH_BYTES = NA_TILES_OFF + NOALLOC_MAX_TILES * sizeof(TileDesc);
+static_assert(NA_SCRATCH_BYTES < 640 * 1024, "no-alloc scratch is meant to stay modest");
+
+}  // namespace
+
+// The fixed device scratch (about 600 KB; every GPU that loads this library
+// holds one copy until the process exits).  In host code this name is only
+// a stand-in for the symbol: its device address comes from
+// cudaGetSymbolAddress, once per device, in noalloc_setup.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NA_SCRATCH_BYTES];
+
+namespace {
+
+struct NoAllocDevice {
+  bool ready = false;
+  unsigned char* scratch = nullptr;   // device address of g_noalloc_scratch on this device
+  logmel_plan plan;                   // default front-end; tables and status word point into scratch
+};
+
+NoAllocDevice g_noalloc[NOALLOC_MAX_DEVICES];
+std::mutex g_noalloc_mu;                                  // set-up and the host metadata buffer
+alignas(16) unsigned char g_noalloc_meta[NA_META_CAP];    // host side of the metadata copy
+
+}  // namespace
+
+// Once per device, with that device current: look up the scratch address,
+// build the default tables and filterbank on the host, upload the tables
+// with a synchronous copy and set the kernel's shared-memory attribute.
+static logmel_status noalloc_setup(int dev, NoAllocDevice& d) {
+  void* sym = nullptr;
+  CK(cudaGetSymbolAddress(&sym, g_noalloc_scratch));
+  logmel_plan& p = d.plan;
+  p.sr = 16000;
+  p.n_fft = NFFT;
+  p.hop = HOP;
+  p.n_mels = 128;
+  p.fmin = 0.f;
+  p.fmax = 8000.f;
+  p.device = dev;
+  Tables t;
+  logmel_status st = build_tables(&t);
+  if (st == LOGMEL_OK) st = build_mel(&p);
+  if (st != LOGMEL_OK) return st;
+  if (!p.default_mel) return LOGMEL_ERR_UNSUPPORTED;   // the compiled layout is this filterbank
+  int sms = 0, max_smem = 0;
+  CK(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  CK(cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
+  shape_launch(p.off, OFFLINE_SPAN_BLOCKS, p.n_mels, max_smem);
+  shape_launch(p.str, STREAM_SPAN_BLOCKS, p.n_mels, max_smem);
+  st = setup_kernel<true>(&p, sms);
+  if (st != LOGMEL_OK) return st;
+  unsigned char* base = static_cast<unsigned char*>(sym);
+  CK(cudaMemcpy(base + NA_TABLES_OFF, &t, sizeof(Tables), cudaMemcpyHostToDevice));
+  p.d_tables = reinterpret_cast<Tables*>(base + NA_TABLES_OFF);
+  p.d_status = reinterpret_cast<int*>(base + NA_STATUS_OFF);
+  d.scratch = base;
+  d.ready = true;
+  return LOGMEL_OK;
+}
+
+extern "C" logmel_status logmel_compute_noalloc(const float* pcm, const int64_t* off, int64_t n_utt,
+                                                 float* out, int* device_status, void* stream) {
+  logmel_status st = check_offsets(off, n_utt);
+  if (st != LOGMEL_OK) return st;
+  if (n_utt == 0) return LOGMEL_OK;
+  if (n_utt > NOALLOC_MAX_UTT) return LOGMEL_ERR_NOALLOC_LIMIT;
+  int64_t frames = 0, tiles = 0;
+  for (int64_t u = 0; u < n_utt; ++u) {
+    const int64_t f = frames_of(off[u + 1] - off[u]);
+    frames += f;
+    tiles += (f + TILE - 1) / TILE;
+  }
+  if (frames == 0) return LOGMEL_OK;
+  if (!pcm || !out) return LOGMEL_ERR_INVALID_ARG;
+  if (tiles > NOALLOC_MAX_TILES) return LOGMEL_ERR_NOALLOC_LIMIT;
+  int dev = -1;
+  CK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= NOALLOC_MAX_DEVICES) return LOGMEL_ERR_UNSUPPORTED;
+
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  NoAllocDevice& d = g_noalloc[dev];
+  if (!d.ready) {
+    st = noalloc_setup(dev, d);
+    if (st != LOGMEL_OK) return st;
+  }
+  // ragged index map, as logmel_compute builds it, in the static host buffer;
+  // a copy from pageable memory has consumed its source when it returns
+  const size_t bytes = meta_bytes(n_utt);
+  MetaView hv = meta_view(g_noalloc_meta, n_utt);
+  hv.frame_off[0] = 0;
+  hv.tile_off[0] = 0;
+  for (int64_t u = 0; u <= n_utt; ++u) hv.sample_off[u] = off[u];
+  for (int64_t u = 0; u < n_utt; ++u) {
+    const int64_t f = frames_of(off[u + 1] - off[u]);
+    hv.frame_off[u + 1] = hv.frame_off[u] + f;
+    hv.tile_off[u + 1] = hv.tile_off[u] + (int)((f + TILE - 1) / TILE);
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned char* dmeta = d.scratch + NA_META_OFF;
+  CK(cudaMemcpyAsync(dmeta, g_noalloc_meta, bytes, cudaMemcpyHostToDevice, s));
+  // the status word starts at zero on every call; the tile descriptors are
+  // rewritten by the kernel before it reads them, so they need no clearing
+  int* status = device_status ? device_status : d.plan.d_status;
+  CK(cudaMemsetAsync(status, 0, sizeof(int), s));
+  MetaView dv = meta_view(dmeta, n_utt);
+  Args a{};
+  a.out = out;
+  a.status = status;
+  a.mode = 0;
+  a.tiles = reinterpret_cast<TileDesc*>(d.scratch + NA_TILES_OFF);
+  // the PCM as rows of 160 samples for one-box tile copies, as in logmel_compute
+  const int64_t total = off[n_utt];
+  const int64_t rows = total / HOP;
+  a.tmap_rows = 0;
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (enc && (reinterpret_cast<uintptr_t>(pcm) & 15) == 0 && rows >= 1 && rows < INT32_MAX) {
+    cuuint64_t dims[2] = {(cuuint64_t)HOP, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)HOP * sizeof(float)};
+    cuuint32_t box[2] = {(cuuint32_t)BLK, (cuuint32_t)OFFLINE_SPAN_BLOCKS};
+    cuuint32_t estr[2] = {1, 1};
+    if (enc(&a.tmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(pcm), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+      a.tmap_rows = (int)rows;
+  }
+  a.num_tiles = (int)tiles;
+  a.n_mels = d.plan.n_mels;
+  a.pcm = pcm;
+  a.sample_off = dv.sample_off;
+  a.frame_off = dv.frame_off;
+  a.tile_off = dv.tile_off;
+  a.n_utt = (int)n_utt;
+  if (launch(&d.plan, a, tiles, s) != cudaSuccess) return LOGMEL_ERR_CUDA;
+  return LOGMEL_OK;
+}
