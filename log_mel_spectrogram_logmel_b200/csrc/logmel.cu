@@ -93,6 +93,26 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
+// The output rows as a 2-D tensor [rows][n_mels] for one-box stores of full
+// tiles: the box is orow_floats(n_mels) x 32, matching the staged rows in
+// shared memory; its pad columns lie outside the tensor and are not written.
+// Returns the tensor's rows, or 0 when no map can be made (unaligned base,
+// row size not a multiple of 16 bytes, no encoder).
+int encode_out_map(CUtensorMap* m, float* out, int64_t rows, int n_mels) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc || (reinterpret_cast<uintptr_t>(out) & 15) || rows < 1 || rows >= INT32_MAX || (n_mels * 4) % 16)
+    return 0;
+  cuuint64_t dims[2] = {(cuuint64_t)n_mels, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)n_mels * sizeof(float)};
+  cuuint32_t box[2] = {(cuuint32_t)orow_floats(n_mels), (cuuint32_t)TILE};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, out, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS
+             ? (int)rows
+             : 0;
+}
+
 }  // namespace
 
 struct LaunchCfg {
@@ -125,6 +145,11 @@ struct logmel_plan {
   const float* tmap_pcm = nullptr;
   int64_t tmap_len = -1;
   int tmap_rows = 0;
+  // tensor map of the last offline output buffer (full-tile row stores)
+  CUtensorMap otmap{};
+  const float* otmap_out = nullptr;
+  int64_t otmap_len = -1;
+  int otmap_rows = 0;
 };
 
 struct logmel_stream {
@@ -230,7 +255,8 @@ static logmel_status build_tables(Tables* t) {
 // Triangular filters, linear in Hz between mel-spaced edges, unnormalised
 // (section 2.3 step 4), stored as contiguous nonzero runs per band; weights
 // carry the factor 1/4 of the real split (which yields |2 X|^2).  Also the
-// split of the bands over the mel warps (cost per band = nonzeros + 3).
+// split of the bands over the mel warps (cost per band = nonzeros + 3, bands
+// taken four at a time).
 static logmel_status build_mel(logmel_plan* p) {
   Args& a = p->mel;
   const int nm = p->n_mels;
@@ -268,10 +294,16 @@ static logmel_status build_mel(logmel_plan* p) {
   a.warp_band[0] = 0;
   long run = 0;
   int m = 0;
-  for (int w = 1; w < MEL_WARPS; ++w) {
+  for (int w = 1; w < MEL_WARPS; ++w) {   // four bands at a time
     const long target = total * w / MEL_WARPS;
-    while (m < nm && run + cost[m] / 2 < target) run += cost[m++];
-    a.warp_band[w] = (short)m;
+    while (m < nm) {
+      long c4 = 0;
+      for (int i = m; i < std::min(m + 4, nm); ++i) c4 += cost[i];
+      if (run + c4 / 2 >= target) break;
+      run += c4;
+      m += 4;
+    }
+    a.warp_band[w] = (short)std::min(m, nm);
   }
   a.warp_band[MEL_WARPS] = (short)nm;
   // the unrolled path applies when the structure equals the compiled one
@@ -560,6 +592,15 @@ logmel_status logmel_compute(logmel_plan* p, const float* pcm, const int64_t* of
   }
   a.tmap = p->tmap;
   a.tmap_rows = p->tmap_rows;
+  if (p->default_mel) {
+    if (out != p->otmap_out || frames != p->otmap_len) {
+      p->otmap_out = out;
+      p->otmap_len = frames;
+      p->otmap_rows = encode_out_map(&p->otmap, out, frames, p->n_mels);
+    }
+    a.otmap = p->otmap;
+    a.otmap_rows = p->otmap_rows;
+  }
   a.num_tiles = (int)tiles;
   a.n_mels = p->n_mels;
   a.pcm = pcm;
@@ -928,6 +969,7 @@ extern "C" logmel_status logmel_compute_noalloc(const float* pcm, const int64_t*
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
       a.tmap_rows = (int)rows;
   }
+  a.otmap_rows = encode_out_map(&a.otmap, out, frames, d.plan.n_mels);
   a.num_tiles = (int)tiles;
   a.n_mels = d.plan.n_mels;
   a.pcm = pcm;

@@ -8,10 +8,12 @@
 // Structure (one persistent kernel, 160 threads, tiles of 32 frames; frame
 // slots d and d + 16 form the pair carried by one thread):
 //   stage   each tile's overlapping sample span is copied from HBM once into
-//           shared memory by the bulk-copy (TMA) engine, one copy per
-//           160-sample hop block into 164-float slots (cp.async when the
-//           source is not 16-byte aligned); a half-warp reads 8 frame pairs
-//           x 2 roles, which keeps pass A's strided reads conflict-free
+//           shared memory by the bulk-copy (TMA) engine: one 2-D tensor copy
+//           of 34 rows of 160 samples into 164-float slots when the span
+//           starts on a 160-sample row, else one bulk copy per hop block
+//           (cp.async when the source is not 16-byte aligned); a half-warp
+//           reads 8 frame pairs x 2 roles, so pass A's strided reads are
+//           conflict-free
 //   pass A  real FFT-400 as a complex FFT-200 of z[m] = x[2m] + i x[2m+1]
 //           (window applied on load), Cooley-Tukey 200 = 20 x 10: ten
 //           20-point DFTs per frame (prime-factor 4 x 5, no inner twiddles),
@@ -19,14 +21,16 @@
 //   pass B  twenty 10-point DFTs (prime-factor 2 x 5); a thread owns the two
 //           tasks k1 and 20 - k1, so Z[k] and Z[200 - k] meet in registers and
 //           the real-FFT split X[k] = (A + u_k B) / 2, u_k = -i e^{-2 pi i k/400},
-//           and the power |2 X[k]|^2 need no exchange
-//   mel     lane = frame, warp = group of bands balanced by nonzeros; each
-//           band sums weight * power over its contiguous bins in a fixed order
-//           (fully unrolled for the default 128-band filterbank, weights read
-//           from the kernel's constant parameter bank)
-//   log     ln via __logf, exact floor constant when the energy is < 1e-10
-//   store   rows of n_mels fp32, transposed into dense rows in shared
-//           memory and written by one bulk copy per run of rows
+//           and the power |2 X[k]|^2 need no exchange; power rows are stored
+//           bin-major, one 8-byte store per frame pair and bin
+//   mel     lane = frame, warp = group of bands (multiples of 4) balanced by
+//           nonzeros; each band sums weight * power over its contiguous bins
+//           in a fixed order (fully unrolled for the default 128-band
+//           filterbank, weights as immediates)
+//   log     ln = lg2 * ln 2, clamped below at the fp32 value of ln(1e-10)
+//   store   each frame's row of n_mels fp32 is staged in shared memory by
+//           16-byte stores (four bands) and leaves through one 2-D tensor
+//           copy per full tile, else one bulk copy per row
 // Two frames ride in the two lanes of packed f32x2 arithmetic (add/sub/mul/
 // fma .f32x2), so a frame's arithmetic never depends on its partner frame:
 // a frame gives the same bits whichever tile, slot or partner it lands in,
@@ -51,14 +55,12 @@ constexpr int N2 = 10;
 constexpr int ROLES = 10;             // threads per frame pair in each pass
 constexpr int THREADS = DUOS * ROLES; // 160
 constexpr int BLK = 164;              // smem floats per hop block: 16-byte aligned (bulk copies)
-constexpr int PSTRIDE = NBINS - 2;    // power rows hold bins 1..199 (odd stride: conflict-free)
 constexpr int YROW = N2;              // float4 per pass-A output row
 constexpr int YDUO = N1 * YROW + 1;   // float4 per frame pair (odd: conflict-free by lane = pair)
 constexpr int MAX_GROUPS = 4;
 constexpr int MEL_WARPS = THREADS / 32;   // 5
 constexpr int MAX_MELS = NBINS;
 constexpr int MAX_WEIGHTS = 2 * NBINS;    // each bin feeds at most two triangles
-constexpr int OSTRIDE = TILE + 1;         // staged output [n_mels][33]
 constexpr int CARRY_CAP = NFFT;           // carried samples per stream (< 400)
 
 // ln(1e-10) rounded to fp32: the value written wherever the mel energy is
@@ -105,8 +107,13 @@ struct Args {
   // lands one tile's span in its hop-block slots (columns 160..163 of a box
   // row are outside the tensor and read as zeros: padding)
   CUtensorMap tmap;
-  int tmap_rows;        // rows of the tensor (0: no tensor map)
-  int pad_tm_[3];
+  // offline: the output as a 2-D tensor [rows][n_mels]; an
+  // orow_floats(n_mels) x 32 box stores one full tile's staged rows (the pad
+  // columns fall outside the tensor)
+  CUtensorMap otmap;
+  int tmap_rows;        // rows of the input tensor (0: no tensor map)
+  int otmap_rows;       // rows of the output tensor (0: no tensor map)
+  int pad_tm_[2];
   const Tables* tables;
   TileDesc* tiles;      // offline: per-tile descriptors (written by the kernel's prologue)
   float* out;
@@ -243,8 +250,8 @@ __device__ __forceinline__ cx sel(bool p, const cx& a, const cx& b) {
 // [control block x 2][pass buffer][span region]
 //   control      groups and per-slot rows of the current and the next tile
 //   pass buffer  pass-A output (float4 per complex pair); after pass B has
-//                read it, the power rows [32][199] and the staged output
-//                [n_mels][OSTRIDE]
+//                read it, the power rows [199 bins][32 frame columns] and
+//                the staged output rows [32][orow_floats(n_mels)]
 //   span region  staged samples (the next tile's span is fetched while the
 //                current tile finishes pass B, mel and store)
 // A CTA runs several independent tile groups (named barriers per group), so
@@ -266,22 +273,38 @@ struct __align__(16) Ctl {
 constexpr int TAB_BYTES = (int)((sizeof(Tables) + 127) / 128 * 128);
 constexpr int CTL_BYTES = (int)((sizeof(Ctl) + 127) / 128 * 128);   // span region 128-byte aligned
 constexpr int YBUF_BYTES = DUOS * YDUO * 16;
-constexpr int PROWS_FLOATS = TILE * PSTRIDE;
+constexpr int PROWS_FLOATS = (NBINS - 2) * TILE;   // power rows: bin k (1..199) at row k - 1
 constexpr int OFFLINE_SPAN_BLOCKS = 34;   // 32 frames: 31 * 160 + 400 samples
 constexpr int STREAM_SPAN_BLOCKS = 40;    // 4 groups of up to 8 frames
 static_assert(sizeof(mel_default::WARP_BAND) == sizeof(int) * (MEL_WARPS + 1), "default band split must match the mel warps");
 static_assert(THREADS == GROUP_THREADS, "a tile group is one tile's threads");
 
+// Staged output rows [32 frame slots][orow_floats(n_mels)]: the pitch is 4
+// mod 8 floats, so 16-byte stores by 32 lanes (one row each) hit distinct
+// banks in every quarter warp.
+__host__ __device__ constexpr int orow_floats(int n_mels) {
+  return (n_mels + 3) / 4 * 4 + ((n_mels + 3) / 4 % 2 == 0 ? 4 : 0);
+}
 // Every region starts on a 128-byte boundary: a tensor bulk copy's shared
-// memory destination must be 128-byte aligned.
+// memory address must be 128-byte aligned (the output rows follow the power
+// rows, whose size is a multiple of 128 bytes).
 __host__ __device__ constexpr int ybuf_bytes_for(int n_mels) {
-  return (((PROWS_FLOATS + n_mels * OSTRIDE) * 4 > YBUF_BYTES ? (PROWS_FLOATS + n_mels * OSTRIDE) * 4 : YBUF_BYTES) +
+  return (((PROWS_FLOATS + TILE * orow_floats(n_mels)) * 4 > YBUF_BYTES
+               ? (PROWS_FLOATS + TILE * orow_floats(n_mels)) * 4
+               : YBUF_BYTES) +
           127) / 128 * 128;
 }
+static_assert(PROWS_FLOATS * 4 % 128 == 0, "output rows start 128-byte aligned");
 static_assert(YBUF_BYTES % 128 == 0 && CTL_BYTES % 128 == 0 && TAB_BYTES % 128 == 0, "128-byte aligned regions");
 __host__ __device__ constexpr int group_bytes_for(int span_blocks, int n_mels) {
   return (2 * CTL_BYTES + ybuf_bytes_for(n_mels) + span_blocks * BLK * 4 + 127) / 128 * 128;
 }
+
+// Power-row column of frame slot f for a bin of parity par: the frames d and
+// d + 16 of a pair sit in columns 2d and 2d + 1, and odd bins swap the two
+// column halves (the two roles of a warp write rows of opposite parity, so
+// their 8-byte pair stores hit distinct banks).
+__device__ __forceinline__ int pcol(int f, int par) { return (2 * (f & 15) + (f >> 4)) ^ (16 * par); }
 
 __device__ __forceinline__ void group_sync(int g) {
   asm volatile("bar.sync %0, %1;" ::"r"(g + 1), "r"(GROUP_THREADS) : "memory");
@@ -343,6 +366,12 @@ __device__ __forceinline__ void tensor_load_2d(void* dst, const CUtensorMap* map
 __device__ __forceinline__ void bulk_store(void* dst, const void* src, unsigned bytes) {
   asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n" ::"l"(dst), "r"(smem_addr(src)),
                "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void tensor_store_2d(const CUtensorMap* map, int x, int y, const void* src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];\n" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(smem_addr(src))
                : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
@@ -524,22 +553,26 @@ __device__ __forceinline__ void stage_tile(Ctl& S, float* span, int tid, const A
 }
 
 // ---------------------------------------------------------------------------
-// mel stage: lane = frame slot s, P = that frame's power row (bins 1..199 at
-// P[k - 1]), o = staged output [band][OSTRIDE]
+// mel stage: lane = frame slot f; bin k of that frame's power row is
+// (k odd ? PO : PE)[k * TILE] (PE, PO: the slot's column for even and odd
+// bins); orow = the slot's staged output row
 // ---------------------------------------------------------------------------
-// ln(max(M, 1e-10)) with the exact floor constant below 1e-10; above it the
-// hardware base-2 logarithm times ln 2 (M >= 1e-10 is normal, so flushing
-// subnormal inputs changes nothing).
+// ln(max(M, 1e-10)): the hardware base-2 logarithm times ln 2, clamped below
+// at the fp32 value of ln(1e-10) (M >= 1e-10 is normal, so flushing subnormal
+// inputs to zero changes nothing).
 __device__ __forceinline__ float log_floor(float acc) {
-  float l2;
+  float l2, r;
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(l2) : "f"(acc));
-  return acc < ENERGY_FLOOR ? LOG_FLOOR : l2 * 0.69314718055994531f;
+  // max(ln M, ln 1e-10) = ln max(M, 1e-10); M = 0 gives -inf, hence the
+  // exact floor; a NaN energy stays NaN
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(l2 * 0.69314718055994531f), "f"(LOG_FLOOR));
+  return r;
 }
 
 // Default 128-band layout, unrolled at compile time: bins and weight offsets
-// are constants, the weights come from the constant parameter bank.
-// sum_j W[WO + j] * p[LO + j - KLO] for j < CNT, in order, weights as
-// immediates, p = the warp's bins held in registers
+// are constants and the weights immediates.
+// sum_j W[WO + j] * p[LO + j - KLO] for j < CNT, in order, p = the warp's bins
+// held in registers
 template <int KLO, int LO, int WO, int J, int CNT, int NP>
 struct MelDot {
   static __device__ __forceinline__ float run(const float (&p)[NP], float acc) {
@@ -552,13 +585,25 @@ struct MelDot {
   }
 };
 
+template <int KLO, int M, int NP>
+__device__ __forceinline__ float mel_band(const float (&p)[NP]) {
+  constexpr int lo = mel_default::LO[M], cnt = mel_default::CNT[M], wo = mel_default::WOFF[M];
+  return log_floor(MelDot<KLO, lo, wo, 0, cnt, NP>::run(p, 0.f));
+}
+
+// bands [M, MEND) four at a time, one 16-byte store per four bands
 template <int KLO, int M, int MEND, int NP>
 struct MelBands {
-  static __device__ __forceinline__ void run(const float (&p)[NP], float* __restrict__ o, int s) {
+  static __device__ __forceinline__ void run(const float (&p)[NP], float* __restrict__ orow) {
     if constexpr (M < MEND) {
-      constexpr int lo = mel_default::LO[M], cnt = mel_default::CNT[M], wo = mel_default::WOFF[M];
-      o[M * OSTRIDE + s] = log_floor(MelDot<KLO, lo, wo, 0, cnt, NP>::run(p, 0.f));
-      MelBands<KLO, M + 1, MEND, NP>::run(p, o, s);
+      static_assert(M % 4 == 0 && MEND % 4 == 0, "warp band ranges are multiples of 4");
+      float4 v;
+      v.x = mel_band<KLO, M, NP>(p);
+      v.y = mel_band<KLO, M + 1, NP>(p);
+      v.z = mel_band<KLO, M + 2, NP>(p);
+      v.w = mel_band<KLO, M + 3, NP>(p);
+      *reinterpret_cast<float4*>(orow + M) = v;
+      MelBands<KLO, M + 4, MEND, NP>::run(p, orow);
     }
   }
 };
@@ -579,22 +624,27 @@ __host__ __device__ constexpr int mel_bin_hi(int b0, int b1) {
 }
 
 template <int W>
-__device__ __forceinline__ void mel_default_warp(const float* __restrict__ P, float* __restrict__ o, int s) {
+__device__ __forceinline__ void mel_default_warp(const float* __restrict__ PE, const float* __restrict__ PO,
+                                                 float* __restrict__ orow) {
   constexpr int B0 = mel_default::WARP_BAND[W], B1 = mel_default::WARP_BAND[W + 1];
   constexpr int KLO = mel_bin_lo(B0, B1), KHI = mel_bin_hi(B0, B1), NP = KHI - KLO + 1;
   float p[NP];
 #pragma unroll
-  for (int i = 0; i < NP; ++i) p[i] = P[KLO + i];   // each bin read once
-  MelBands<KLO, B0, B1, NP>::run(p, o, s);
+  for (int i = 0; i < NP; ++i) p[i] = (((KLO + i) & 1) ? PO : PE)[(KLO + i) * TILE];   // each bin read once
+  MelBands<KLO, B0, B1, NP>::run(p, orow);
 }
 
-__device__ __forceinline__ void mel_generic_warp(const Args& a, int w, const float* P, float* o, int s) {
+__device__ __forceinline__ void mel_generic_warp(const Args& a, int w, const float* PE, const float* PO,
+                                                 float* orow) {
   const int mb = a.warp_band[w], me = a.warp_band[w + 1];
   for (int m = mb; m < me; ++m) {
     const int lo = a.mel_lo[m], cnt = a.mel_cnt[m], wo = a.mel_woff[m];
     float acc = 0.f;
-    for (int j = 0; j < cnt; ++j) acc = fmaf(a.mel_w[wo + j], P[lo + j], acc);
-    o[m * OSTRIDE + s] = log_floor(acc);
+    for (int j = 0; j < cnt; ++j) {
+      const int k = lo + j;
+      acc = fmaf(a.mel_w[wo + j], ((k & 1) ? PO : PE)[k * TILE], acc);
+    }
+    orow[m] = log_floor(acc);
   }
 }
 
@@ -659,9 +709,9 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
   float4* const Y = reinterpret_cast<float4*>(gbase + 2 * CTL_BYTES);
   float* const span = reinterpret_cast<float*>(gbase + 2 * CTL_BYTES + a.ybuf_bytes);
   float* const Pbuf = reinterpret_cast<float*>(Y);   // power rows, after pass B has read Y
-  float* const outS = Pbuf + PROWS_FLOATS;           // staged output, after the power rows
+  float* const orows = Pbuf + PROWS_FLOATS;          // staged output rows, after the power rows
+  const int opitch = orow_floats(a.n_mels);
 
-  const int n_mels = a.n_mels;
   int tile = blockIdx.x * G + grp;
   if (tile < a.num_tiles) {
     if (tid == COPY_TID) {
@@ -684,7 +734,7 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
       // the verdict so the whole group takes the same path
       S.copy_ok = S.tma ? mbar_wait(&S.bar, S.bar_parity, 1 << 16) : 1;
     }
-    if (tid == 0) bulk_wait_read();   // the previous tile's bulk row copies have read smem
+    if (warp == 0) bulk_wait_read();   // the previous tile's bulk row copies have read smem
     asm volatile("cp.async.wait_all;\n" ::: "memory");
     group_sync(grp);   // this tile's span is staged; the previous tile's rows are stored
     if (!S.copy_ok) {   // a bulk copy never completed: flag it and stop this group
@@ -768,8 +818,9 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
       dft10(za);
       dft10(zb);
       // za[pos10(k2)] = Z[ka + 20 k2], zb[pos10(k2)] = Z[kb + 20 k2].
-      float* PA = Pbuf + d * PSTRIDE - 1;            // frame slot d, bin k at PA[k]
-      float* PB = Pbuf + (d + DUOS) * PSTRIDE - 1;   // frame slot d + 16
+      // bin k of slots d and d + 16 at PP[k * TILE] (both bins k and 200 - k
+      // of a role have the role's parity)
+      float* PP = Pbuf - TILE + pcol(d, r & 1);
       if (warp != 0) {
         // roles 2..9: slot j couples Z[k], k = r + 20 j, with Z[200 - k] = zb[9 - j]
 #pragma unroll
@@ -777,10 +828,8 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
           const int k = r + 20 * j;
           float2 pk, pm;
           split_power(tab, za[pos10(j)], zb[pos10(9 - j)], k, pk, pm);
-          PA[k] = pk.x;
-          PB[k] = pk.y;
-          PA[200 - k] = pm.x;
-          PB[200 - k] = pm.y;
+          *reinterpret_cast<float2*>(PP + k * TILE) = pk;
+          *reinterpret_cast<float2*>(PP + (200 - k) * TILE) = pm;
         }
       } else {
         // roles 0 and 1 share this warp; role 0 owns the self-paired tasks
@@ -797,18 +846,15 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
           float2 pk, pm;
           split_power(tab, zk, zm, k, pk, pm);
           if (k > 0) {
-            PA[k] = pk.x;
-            PB[k] = pk.y;
-            PA[200 - k] = pm.x;
-            PB[200 - k] = pm.y;
+            *reinterpret_cast<float2*>(PP + k * TILE) = pk;
+            *reinterpret_cast<float2*>(PP + (200 - k) * TILE) = pm;
           }
         }
         if (r0) {
           const cx z = za[pos10(5)];
           const float2 tr = add2(z.re, z.re), ti = add2(z.im, z.im);
           const float2 p = fma2(ti, ti, mul2(tr, tr));
-          PA[100] = p.x;
-          PB[100] = p.y;
+          *reinterpret_cast<float2*>(PP + 100 * TILE) = p;
         }
       }
     }
@@ -816,71 +862,49 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
 
     // ---- mel + log: warp = band group, lane = frame slot ------------------
     {
-      const float* P = Pbuf + lane * PSTRIDE - 1;
+      const float* PE = Pbuf - TILE + pcol(lane, 0);
+      const float* PO = Pbuf - TILE + pcol(lane, 1);
+      float* orow = orows + lane * opitch;
       if constexpr (kDefaultMel) {
         switch (warp) {
-          case 0: mel_default_warp<0>(P, outS, lane); break;
-          case 1: mel_default_warp<1>(P, outS, lane); break;
-          case 2: mel_default_warp<2>(P, outS, lane); break;
-          case 3: mel_default_warp<3>(P, outS, lane); break;
-          default: mel_default_warp<4>(P, outS, lane); break;
+          case 0: mel_default_warp<0>(PE, PO, orow); break;
+          case 1: mel_default_warp<1>(PE, PO, orow); break;
+          case 2: mel_default_warp<2>(PE, PO, orow); break;
+          case 3: mel_default_warp<3>(PE, PO, orow); break;
+          default: mel_default_warp<4>(PE, PO, orow); break;
         }
       } else {
-        mel_generic_warp(a, warp, P, outS, lane);
+        mel_generic_warp(a, warp, PE, PO, orow);
       }
     }
+    if (a.bulk_store) fence_async_smem();   // the staged rows precede the bulk copies reading them
     group_sync(grp);
 
-    // ---- store: rows of n_mels fp32, one warp per row ---------------------
+    // ---- store: the staged rows of the tile's frames ---------------------
     {
-      const float* o = outS;
       const int ns = S.nslots;
-      if constexpr (kDefaultMel) {
-        constexpr int NM = mel_default::N_MELS;
-        if (a.bulk_store) {
-          // transpose into dense rows (in the dead power-row region), then one
-          // bulk copy per group of consecutive rows
-          float* dense = Pbuf;
-#pragma unroll
-          for (int rr = 0; rr < (TILE + MEL_WARPS - 1) / MEL_WARPS; ++rr) {
-            const int s = warp + MEL_WARPS * rr;
-            if (s < ns) {
-              const float* src = o + lane * OSTRIDE + s;
-#pragma unroll
-              for (int q = 0; q < NM / 32; ++q) dense[s * NM + lane + 32 * q] = src[32 * q * OSTRIDE];
-            }
+      if (a.bulk_store) {
+        // one tensor copy for a full offline tile (the box's pad columns lie
+        // outside the output tensor and are not written), else one bulk copy
+        // per row, issued by the lanes of warp 0
+        if (warp == 0) {
+          if (a.mode == 0 && ns == TILE && a.otmap_rows > 0) {
+            if (lane == 0) tensor_store_2d(&a.otmap, 0, (int)S.groups[0].out_row, orows);
+          } else if (lane < ns) {
+            bulk_store(a.out + slot_row(S, lane) * a.n_mels, orows + lane * opitch, (unsigned)a.n_mels * 4u);
           }
-          fence_async_smem();
-          group_sync(grp);
-          if (tid == 0) {
-            for (int gi = 0; gi < S.ngroups; ++gi) {
-              const Group& g = S.groups[gi];
-              if (g.nframes > 0)
-                bulk_store(a.out + g.out_row * NM, dense + g.slot0 * NM, (unsigned)g.nframes * NM * 4u);
-            }
-            bulk_commit();
-          }
-        } else {
-#pragma unroll
-          for (int rr = 0; rr < (TILE + MEL_WARPS - 1) / MEL_WARPS; ++rr) {
-            const int s = warp + MEL_WARPS * rr;
-            if (s < ns) {
-              float* row = a.out + slot_row(S, s) * NM + lane;
-              const float* src = o + lane * OSTRIDE + s;
-#pragma unroll
-              for (int q = 0; q < NM / 32; ++q) row[32 * q] = src[32 * q * OSTRIDE];
-            }
-          }
+          bulk_commit();
         }
       } else {
         for (int s = warp; s < ns; s += MEL_WARPS) {
-          float* row = a.out + slot_row(S, s) * n_mels;
-          for (int m = lane; m < n_mels; m += 32) row[m] = o[m * OSTRIDE + s];
+          float* row = a.out + slot_row(S, s) * a.n_mels;
+          const float* src = orows + s * opitch;
+          for (int m = lane; m < a.n_mels; m += 32) row[m] = src[m];
         }
       }
     }
   }
-  if (tid == 0) asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");   // rows written before exit
+  if (warp == 0) asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");   // rows written before exit
 }
 
 }  // namespace logmel
