@@ -101,11 +101,12 @@ logmel_status logmel_frame_offsets(const logmel_plan* plan, const int64_t* offse
  *            total_frames = sum of logmel_num_frames over utterances; the
  *            rows of utterance u start at frame_offsets[u]
  * Utterances shorter than n_fft contribute no rows and no error.  The call
- * copies a few bytes of tile metadata host->device on `stream` (from a
- * pinned ring owned by the plan) and launches one kernel; it does not
- * synchronise unless the plan's scratch must grow (first call with a larger
- * batch), which synchronises the device.  n_utt == 0 or total_frames == 0
- * is a no-op. */
+ * launches one kernel.  For n_utt <= 256 the per-utterance offsets travel in
+ * the launch parameters; larger batches first copy them host->device on
+ * `stream` (from a pinned ring owned by the plan).  It does not synchronise
+ * unless the plan's scratch must grow (first call with a larger batch of
+ * more than 256 utterances), which synchronises the device.  n_utt == 0 or
+ * total_frames == 0 is a no-op. */
 logmel_status logmel_compute(logmel_plan* plan, const float* pcm, const int64_t* offsets,
                              int64_t n_utt, float* out, void* stream);
 
@@ -196,9 +197,10 @@ logmel_status logmel_stream_reset(logmel_stream* st, int stream_id, void* stream
  * contents: calls whose work overlaps on the GPU (two streams, or two host
  * threads without ordering) race on it and may return wrong output; order
  * them on one stream or with events.  Host-side, calls are serialised by a
- * lock.  Each call copies its metadata host->device from a static host
- * buffer with cudaMemcpyAsync and launches one kernel; no device or pinned
- * memory is allocated or freed. */
+ * lock.  Each call clears the status word and launches one kernel; batches
+ * of more than 256 utterances first copy their metadata host->device from a
+ * static host buffer with cudaMemcpyAsync.  No device or pinned memory is
+ * allocated or freed. */
 logmel_status logmel_compute_noalloc(const float* pcm, const int64_t* offsets, int64_t n_utt,
                                      float* out, int* device_status, void* stream);
 

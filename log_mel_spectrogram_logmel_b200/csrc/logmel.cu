@@ -533,42 +533,59 @@ logmel_status logmel_compute(logmel_plan* p, const float* pcm, const int64_t* of
   if (frames == 0) return LOGMEL_OK;
   if (!pcm || !out) return LOGMEL_ERR_INVALID_ARG;
   if (tiles >= INT32_MAX || frames >= INT32_MAX) return LOGMEL_ERR_INPUT_TOO_LONG;
-  const size_t bytes = meta_bytes(n_utt);
-  st = ensure_meta(p, bytes);
-  if (st != LOGMEL_OK) return st;
-  if ((size_t)tiles > p->tiles_cap) {
-    CK(cudaDeviceSynchronize());
-    CK(cudaFree(p->d_tiles));
-    p->d_tiles = nullptr;
-    const size_t cap = std::max<size_t>((size_t)tiles, 1024);
-    if (cudaMalloc(&p->d_tiles, cap * sizeof(TileDesc)) != cudaSuccess) {
-      p->tiles_cap = 0;
-      return LOGMEL_ERR_OOM;
-    }
-    p->tiles_cap = cap;
-  }
-  PinnedSlot& slot = p->ring[p->ring_next];
-  p->ring_next = (p->ring_next + 1) % RING;
-  if (slot.used) CK(cudaEventSynchronize(slot.done));
-  MetaView hv = meta_view(slot.host, n_utt);
-  hv.frame_off[0] = 0;
-  hv.tile_off[0] = 0;
-  for (int64_t u = 0; u <= n_utt; ++u) hv.sample_off[u] = off[u];
-  for (int64_t u = 0; u < n_utt; ++u) {
-    const int64_t f = frames_of(off[u + 1] - off[u]);
-    hv.frame_off[u + 1] = hv.frame_off[u] + f;
-    hv.tile_off[u + 1] = hv.tile_off[u] + (int)((f + TILE - 1) / TILE);
-  }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  CK(cudaMemcpyAsync(p->d_meta, slot.host, bytes, cudaMemcpyHostToDevice, s));
-  CK(cudaEventRecord(slot.done, s));
-  slot.used = true;
-  MetaView dv = meta_view(p->d_meta, n_utt);
   Args a{};
+  if (n_utt <= INLINE_UTT) {
+    // small batches: the ragged index map travels in the launch parameters,
+    // and the kernel finds each tile's utterance there (no copy, no scratch)
+    a.meta_inline = 1;
+    a.im_frame_off[0] = 0;
+    a.im_tile_off[0] = 0;
+    for (int64_t u = 0; u <= n_utt; ++u) a.im_sample_off[u] = off[u];
+    for (int64_t u = 0; u < n_utt; ++u) {
+      const int64_t f = frames_of(off[u + 1] - off[u]);
+      a.im_frame_off[u + 1] = a.im_frame_off[u] + (int)f;
+      a.im_tile_off[u + 1] = a.im_tile_off[u] + (int)((f + TILE - 1) / TILE);
+    }
+  } else {
+    const size_t bytes = meta_bytes(n_utt);
+    st = ensure_meta(p, bytes);
+    if (st != LOGMEL_OK) return st;
+    if ((size_t)tiles > p->tiles_cap) {
+      CK(cudaDeviceSynchronize());
+      CK(cudaFree(p->d_tiles));
+      p->d_tiles = nullptr;
+      const size_t cap = std::max<size_t>((size_t)tiles, 1024);
+      if (cudaMalloc(&p->d_tiles, cap * sizeof(TileDesc)) != cudaSuccess) {
+        p->tiles_cap = 0;
+        return LOGMEL_ERR_OOM;
+      }
+      p->tiles_cap = cap;
+    }
+    PinnedSlot& slot = p->ring[p->ring_next];
+    p->ring_next = (p->ring_next + 1) % RING;
+    if (slot.used) CK(cudaEventSynchronize(slot.done));
+    MetaView hv = meta_view(slot.host, n_utt);
+    hv.frame_off[0] = 0;
+    hv.tile_off[0] = 0;
+    for (int64_t u = 0; u <= n_utt; ++u) hv.sample_off[u] = off[u];
+    for (int64_t u = 0; u < n_utt; ++u) {
+      const int64_t f = frames_of(off[u + 1] - off[u]);
+      hv.frame_off[u + 1] = hv.frame_off[u] + f;
+      hv.tile_off[u + 1] = hv.tile_off[u] + (int)((f + TILE - 1) / TILE);
+    }
+    CK(cudaMemcpyAsync(p->d_meta, slot.host, bytes, cudaMemcpyHostToDevice, s));
+    CK(cudaEventRecord(slot.done, s));
+    slot.used = true;
+    MetaView dv = meta_view(p->d_meta, n_utt);
+    a.sample_off = dv.sample_off;
+    a.frame_off = dv.frame_off;
+    a.tile_off = dv.tile_off;
+    a.tiles = p->d_tiles;
+  }
   a.out = out;
   a.status = p->d_status;
   a.mode = 0;
-  a.tiles = p->d_tiles;
   // the PCM as rows of 160 samples for one-box tile copies (16-byte aligned
   // base and at least one full row); the box is 164 x 34: columns 160..163
   // are outside the tensor and arrive as zeros
@@ -604,9 +621,6 @@ logmel_status logmel_compute(logmel_plan* p, const float* pcm, const int64_t* of
   a.num_tiles = (int)tiles;
   a.n_mels = p->n_mels;
   a.pcm = pcm;
-  a.sample_off = dv.sample_off;
-  a.frame_off = dv.frame_off;
-  a.tile_off = dv.tile_off;
   a.n_utt = (int)n_utt;
   if (launch(p, a, tiles, s) != cudaSuccess) return LOGMEL_ERR_CUDA;
   return LOGMEL_OK;
@@ -929,31 +943,48 @@ extern "C" logmel_status logmel_compute_noalloc(const float* pcm, const int64_t*
     st = noalloc_setup(dev, d);
     if (st != LOGMEL_OK) return st;
   }
-  // ragged index map, as logmel_compute builds it, in the static host buffer;
-  // a copy from pageable memory has consumed its source when it returns
-  const size_t bytes = meta_bytes(n_utt);
-  MetaView hv = meta_view(g_noalloc_meta, n_utt);
-  hv.frame_off[0] = 0;
-  hv.tile_off[0] = 0;
-  for (int64_t u = 0; u <= n_utt; ++u) hv.sample_off[u] = off[u];
-  for (int64_t u = 0; u < n_utt; ++u) {
-    const int64_t f = frames_of(off[u + 1] - off[u]);
-    hv.frame_off[u + 1] = hv.frame_off[u] + f;
-    hv.tile_off[u + 1] = hv.tile_off[u] + (int)((f + TILE - 1) / TILE);
-  }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  unsigned char* dmeta = d.scratch + NA_META_OFF;
-  CK(cudaMemcpyAsync(dmeta, g_noalloc_meta, bytes, cudaMemcpyHostToDevice, s));
+  Args a{};
+  if (n_utt <= INLINE_UTT) {
+    // the ragged index map in the launch parameters, as logmel_compute does
+    a.meta_inline = 1;
+    a.im_frame_off[0] = 0;
+    a.im_tile_off[0] = 0;
+    for (int64_t u = 0; u <= n_utt; ++u) a.im_sample_off[u] = off[u];
+    for (int64_t u = 0; u < n_utt; ++u) {
+      const int64_t f = frames_of(off[u + 1] - off[u]);
+      a.im_frame_off[u + 1] = a.im_frame_off[u] + (int)f;
+      a.im_tile_off[u + 1] = a.im_tile_off[u] + (int)((f + TILE - 1) / TILE);
+    }
+  } else {
+    // larger batches: the index map in the static host buffer, copied into
+    // the scratch (a copy from pageable memory has consumed its source when
+    // it returns); the kernel writes the tile descriptors into the scratch
+    const size_t bytes = meta_bytes(n_utt);
+    MetaView hv = meta_view(g_noalloc_meta, n_utt);
+    hv.frame_off[0] = 0;
+    hv.tile_off[0] = 0;
+    for (int64_t u = 0; u <= n_utt; ++u) hv.sample_off[u] = off[u];
+    for (int64_t u = 0; u < n_utt; ++u) {
+      const int64_t f = frames_of(off[u + 1] - off[u]);
+      hv.frame_off[u + 1] = hv.frame_off[u] + f;
+      hv.tile_off[u + 1] = hv.tile_off[u] + (int)((f + TILE - 1) / TILE);
+    }
+    unsigned char* dmeta = d.scratch + NA_META_OFF;
+    CK(cudaMemcpyAsync(dmeta, g_noalloc_meta, bytes, cudaMemcpyHostToDevice, s));
+    MetaView dv = meta_view(dmeta, n_utt);
+    a.sample_off = dv.sample_off;
+    a.frame_off = dv.frame_off;
+    a.tile_off = dv.tile_off;
+    a.tiles = reinterpret_cast<TileDesc*>(d.scratch + NA_TILES_OFF);
+  }
   // the status word starts at zero on every call; the tile descriptors are
   // rewritten by the kernel before it reads them, so they need no clearing
   int* status = device_status ? device_status : d.plan.d_status;
   CK(cudaMemsetAsync(status, 0, sizeof(int), s));
-  MetaView dv = meta_view(dmeta, n_utt);
-  Args a{};
   a.out = out;
   a.status = status;
   a.mode = 0;
-  a.tiles = reinterpret_cast<TileDesc*>(d.scratch + NA_TILES_OFF);
   // the PCM as rows of 160 samples for one-box tile copies, as in logmel_compute
   const int64_t total = off[n_utt];
   const int64_t rows = total / HOP;
@@ -973,9 +1004,6 @@ extern "C" logmel_status logmel_compute_noalloc(const float* pcm, const int64_t*
   a.num_tiles = (int)tiles;
   a.n_mels = d.plan.n_mels;
   a.pcm = pcm;
-  a.sample_off = dv.sample_off;
-  a.frame_off = dv.frame_off;
-  a.tile_off = dv.tile_off;
   a.n_utt = (int)n_utt;
   if (launch(&d.plan, a, tiles, s) != cudaSuccess) return LOGMEL_ERR_CUDA;
   return LOGMEL_OK;

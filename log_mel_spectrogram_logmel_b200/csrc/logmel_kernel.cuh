@@ -62,6 +62,7 @@ constexpr int MEL_WARPS = THREADS / 32;   // 5
 constexpr int MAX_MELS = NBINS;
 constexpr int MAX_WEIGHTS = 2 * NBINS;    // each bin feeds at most two triangles
 constexpr int CARRY_CAP = NFFT;           // carried samples per stream (< 400)
+constexpr int INLINE_UTT = 256;           // offline batches up to this size carry their metadata in the parameters
 
 // ln(1e-10) rounded to fp32: the value written wherever the mel energy is
 // below 1e-10 (section 2.3 step 5's floor).
@@ -131,6 +132,7 @@ struct Args {
   const int64_t* frame_off;    // [n_utt + 1]
   const int* tile_off;         // [n_utt + 1]
   int n_utt;
+  int meta_inline;             // 1: the metadata is in im_* below (no device copy)
   // streaming
   float* carry;                // [n_streams][CARRY_CAP]
   int* carry_len;              // [n_streams]
@@ -150,6 +152,11 @@ struct Args {
   short mel_cnt[MAX_MELS];     // contiguous nonzero bins
   short mel_woff[MAX_MELS];    // offset into mel_w
   short warp_band[MEL_WARPS + 1];
+  // offline metadata of batches of up to INLINE_UTT utterances, carried in
+  // the launch itself (no host-to-device copy before the kernel)
+  int64_t im_sample_off[INLINE_UTT + 1];
+  int im_frame_off[INLINE_UTT + 1];
+  int im_tile_off[INLINE_UTT + 1];
 };
 
 enum DeviceStatus : int { STATUS_OK = 0, STATUS_SPAN_OVERFLOW = 1, STATUS_SLOT_OVERFLOW = 2, STATUS_COPY_TIMEOUT = 3 };
@@ -269,6 +276,7 @@ struct __align__(16) Ctl {
   int bar_parity;           // phase of bar to wait for
   int copy_ok;              // the waiting thread's verdict on the bulk copies (0: timed out)
   int tmap_row;             // tensor row of the span's first sample (tma == 2)
+  TileDesc pending;         // offline: the descriptor of the group's tile after next
 };
 constexpr int TAB_BYTES = (int)((sizeof(Tables) + 127) / 128 * 128);
 constexpr int CTL_BYTES = (int)((sizeof(Ctl) + 127) / 128 * 128);   // span region 128-byte aligned
@@ -404,7 +412,8 @@ __device__ __forceinline__ int64_t slot_row(const Ctl& S, int t) {
   return r;
 }
 
-// Offline tile descriptor: binary search of the tile's utterance.
+// Offline tile descriptor: binary search of the tile's utterance in the
+// device metadata.
 __device__ TileDesc offline_desc(const Args& a, int tile) {
   int lo = 0, hi = a.n_utt - 1;   // last u with tile_off[u] <= tile
   while (lo < hi) {
@@ -419,6 +428,26 @@ __device__ TileDesc offline_desc(const Args& a, int tile) {
   t.out_row = (int)(a.frame_off[u] + f0);
   t.nframes = (int)min64(TILE, nfr - f0);
   return t;
+}
+// The same from the metadata carried in the parameters.
+__device__ __noinline__ TileDesc inline_desc(const Args& a, int tile) {
+  int lo = 0, hi = a.n_utt - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (a.im_tile_off[mid] <= tile) lo = mid; else hi = mid - 1;
+  }
+  const int u = lo;
+  const int f0 = (tile - a.im_tile_off[u]) * TILE;
+  TileDesc t;
+  t.src = a.im_sample_off[u] + (int64_t)f0 * HOP;
+  t.out_row = a.im_frame_off[u] + f0;
+  t.nframes = min(TILE, a.im_frame_off[u + 1] - a.im_frame_off[u] - f0);
+  return t;
+}
+// Descriptor of offline tile t: searched in the parameters, or written by
+// the prologue into the descriptor scratch.
+__device__ __forceinline__ TileDesc tile_desc(const Args& a, int t) {
+  return a.meta_inline ? inline_desc(a, t) : a.tiles[t];
 }
 
 __device__ void setup_offline(Ctl& S, const Args& a, const TileDesc& t, const float* span) {
@@ -687,7 +716,7 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
     float4* dst = reinterpret_cast<float4*>(smem_raw);
     for (int i = threadIdx.x; i < (int)(sizeof(Tables) / 16); i += blockDim.x) dst[i] = src[i];
   }
-  if (a.mode == 0) {  // offline: this CTA's tile descriptors, searched in parallel
+  if (a.mode == 0 && !a.meta_inline) {  // offline: this CTA's tile descriptors, searched in parallel
     const int rounds = (a.num_tiles + stride - 1) / stride;
     for (int j = threadIdx.x; j < rounds * G; j += blockDim.x) {
       const int t = blockIdx.x * G + (j % G) + (j / G) * stride;
@@ -715,20 +744,21 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
   int tile = blockIdx.x * G + grp;
   if (tile < a.num_tiles) {
     if (tid == COPY_TID) {
-      if (a.mode == 0) setup_offline(*ctl0, a, a.tiles[tile], span);
+      if (a.mode == 0) setup_offline(*ctl0, a, tile_desc(a, tile), span);
       else setup_stream(*ctl0, a, tile);
       if (ctl0->tma) ctl0->bar_parity = (armed0++) & 1;
     }
     group_sync(grp);
     stage_tile(*ctl0, span, tid, a);
+    if (tid == COPY_TID && a.mode == 0 && tile + stride < a.num_tiles) ctl0->pending = tile_desc(a, tile + stride);
   }
   int cur = 0;
   for (; tile < a.num_tiles; tile += stride, cur ^= 1) {
     Ctl& S = cur ? *ctl1 : *ctl0;
     Ctl& N = cur ? *ctl0 : *ctl1;
     const int next = tile + stride;
-    TileDesc nd;
-    if (tid == COPY_TID && a.mode == 0 && next < a.num_tiles) nd = a.tiles[next];   // used after pass A
+    TileDesc nd;   // the next tile's descriptor (used after pass A)
+    if (tid == COPY_TID && a.mode == 0 && next < a.num_tiles) nd = ctl0->pending;
     if (tid == COPY_TID) {
       // one thread waits for the bulk copies (bounded: ~65 ms), and publishes
       // the verdict so the whole group takes the same path
@@ -903,6 +933,9 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
         }
       }
     }
+    // the descriptor of this group's tile after next, found while warp 0
+    // issues the row copies (used after the next tile's pass A)
+    if (tid == COPY_TID && a.mode == 0 && next + stride < a.num_tiles) ctl0->pending = tile_desc(a, next + stride);
   }
   if (warp == 0) asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");   // rows written before exit
 }

@@ -48,6 +48,23 @@ def test_ragged_batch_small_full_compare(plan):
     check_against_oracle(g, L, M)
 
 
+def test_batch_beyond_inline_metadata(plan):
+    """More than 256 utterances: the ragged index map goes to the device by a
+    copy and the tile descriptors through the kernel's scratch, instead of
+    travelling in the launch parameters.  Both routes give the same bits."""
+    lengths = np.random.default_rng(71).integers(200, 9000, 300)
+    pcm, off = W.ragged_batch(lengths=lengths, seed0=5000)
+    g = _run(plan, pcm, off)
+    L, M = O.log_mel_batch(pcm, off, return_energy=True)
+    check_against_oracle(g, L, M)
+    # the same audio as two batches of 150 utterances (parameter route)
+    h = 150
+    first = _run(plan, pcm[:off[h]], off[:h + 1])
+    second = _run(plan, pcm[off[h]:], off[h:] - off[h])
+    both = np.concatenate([first, second])
+    assert np.array_equal(both.view(np.int32), g.view(np.int32))
+
+
 def _sample_rows(fo, n_random, seed):
     rng = np.random.default_rng(seed)
     rows = set(rng.integers(0, fo[-1], n_random).tolist())
