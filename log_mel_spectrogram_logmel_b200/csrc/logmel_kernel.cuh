@@ -259,8 +259,9 @@ __device__ __forceinline__ cx sel(bool p, const cx& a, const cx& b) {
 //   pass buffer  pass-A output (float4 per complex pair); after pass B has
 //                read it, the power rows [199 bins][32 frame columns] and
 //                the staged output rows [32][orow_floats(n_mels)]
-//   span region  staged samples (the next tile's span is fetched while the
-//                current tile finishes pass B, mel and store)
+//   span region  staged samples (the next tile's span is fetched as soon as
+//                pass A has read the current one: during pass B, mel and
+//                store)
 // A CTA runs several independent tile groups (named barriers per group), so
 // the tables are held once per CTA.  Offline tiles need 34 hop blocks of
 // span, streaming tiles with four groups 40.
@@ -828,6 +829,10 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
     }
     group_sync(grp);
 
+    // every thread has finished reading the span (its values were consumed
+    // before the barrier above): fetch the next tile's span meanwhile
+    if (next < a.num_tiles) stage_tile(N, span, tid, a);
+
     // ---- pass B: 10-point DFTs over m2, real split, power -----------------
     {
       const int r = role;
@@ -842,11 +847,9 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
         za[m2] = cx{make_float2(va.x, va.y), make_float2(va.z, va.w)};
         zb[m2] = cx{make_float2(vb.x, vb.y), make_float2(vb.z, vb.w)};
       }
-      fence_async_smem();  // this thread's span reads precede the bulk copies into it
-      group_sync(grp);   // rows held in registers: power rows may overwrite Y; span is free
-      if (next < a.num_tiles) stage_tile(N, span, tid, a);   // fetch the next tile meanwhile
       dft10(za);
       dft10(zb);
+      group_sync(grp);   // every thread holds its rows: power rows may overwrite Y
       // za[pos10(k2)] = Z[ka + 20 k2], zb[pos10(k2)] = Z[kb + 20 k2].
       // bin k of slots d and d + 16 at PP[k * TILE] (both bins k and 200 - k
       // of a role have the role's parity)
