@@ -275,7 +275,7 @@ struct __align__(16) Ctl {
   int nslots;
   int tma;                  // 1: per-block bulk copies, 2: one tensor copy (wait on bar)
   int bar_parity;           // phase of bar to wait for
-  int copy_ok;              // the waiting thread's verdict on the bulk copies (0: timed out)
+  int copy_ok;              // verdict on the bulk copies (0: a thread's bounded wait gave up)
   int tmap_row;             // tensor row of the span's first sample (tma == 2)
   TileDesc pending;         // offline: the descriptor of the group's tile after next
 };
@@ -748,6 +748,7 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
       if (a.mode == 0) setup_offline(*ctl0, a, tile_desc(a, tile), span);
       else setup_stream(*ctl0, a, tile);
       if (ctl0->tma) ctl0->bar_parity = (armed0++) & 1;
+      ctl0->copy_ok = 1;
     }
     group_sync(grp);
     stage_tile(*ctl0, span, tid, a);
@@ -760,19 +761,17 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
     const int next = tile + stride;
     TileDesc nd;   // the next tile's descriptor (used after pass A)
     if (tid == COPY_TID && a.mode == 0 && next < a.num_tiles) nd = ctl0->pending;
-    if (tid == COPY_TID) {
-      // one thread waits for the bulk copies (bounded: ~65 ms), and publishes
-      // the verdict so the whole group takes the same path
-      S.copy_ok = S.tma ? mbar_wait(&S.bar, S.bar_parity, 1 << 16) : 1;
+    // This tile's span: bulk copies complete on the mbarrier, which every
+    // thread polls (bounded: ~65 ms) before it reads the span; a thread that
+    // gives up clears the verdict, which the whole group reads after the
+    // barrier in pass A.  Per-thread cp.async copies need a barrier to be
+    // seen by the other threads.
+    if (S.tma) {
+      if (!mbar_wait(&S.bar, S.bar_parity, 1 << 16)) S.copy_ok = 0;
+    } else {
+      asm volatile("cp.async.wait_all;\n" ::: "memory");
+      group_sync(grp);
     }
-    if (warp == 0) bulk_wait_read();   // the previous tile's bulk row copies have read smem
-    asm volatile("cp.async.wait_all;\n" ::: "memory");
-    group_sync(grp);   // this tile's span is staged; the previous tile's rows are stored
-    if (!S.copy_ok) {   // a bulk copy never completed: flag it and stop this group
-      if (tid == COPY_TID) atomicExch(a.status, STATUS_COPY_TIMEOUT);
-      break;
-    }
-    if (S.tma) mbar_wait(&S.bar, S.bar_parity, 1 << 16);   // completed: acquires the copied span
     const int ng = S.ngroups;
 
     // ---- streaming: write each owned stream's new carry from the span -----
@@ -806,19 +805,29 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
         z[m1].im = make_float2(xa.y * w.y, xb.y * w.y);
       }
       dft20(z);
+#pragma unroll
+      for (int k1 = 1; k1 < N1; ++k1) {
+        cx& v = z[pos20(k1)];
+        const float4 t = tab.w400[2 * m2 * k1];   // e^{-2 pi i m2 k1 / 200} = c - i s
+        const float2 c = make_float2(t.x, t.y), sn = make_float2(t.z, t.w);
+        // (re + i im)(c - i s) = (re c + im s) + i (im c - re s)
+        const float2 re = fma2(v.im, sn, mul2(v.re, c));
+        const float2 im = sub2(mul2(v.im, c), mul2(v.re, sn));
+        v.re = re;
+        v.im = im;
+      }
+      // the previous tile's mel stage and row copies are done with the pass
+      // buffer before it is overwritten, and every copy verdict is in
+      if (warp == 0) bulk_wait_read();
+      group_sync(grp);
+      if (!S.copy_ok) {   // a bulk copy never completed: flag it and stop this group
+        if (tid == COPY_TID) atomicExch(a.status, STATUS_COPY_TIMEOUT);
+        break;
+      }
       float4* yrow = Y + d * YDUO + m2;
 #pragma unroll
       for (int k1 = 0; k1 < N1; ++k1) {
-        cx v = z[pos20(k1)];
-        if (k1 > 0) {
-          const float4 t = tab.w400[2 * m2 * k1];   // e^{-2 pi i m2 k1 / 200} = c - i s
-          const float2 c = make_float2(t.x, t.y), sn = make_float2(t.z, t.w);
-          // (re + i im)(c - i s) = (re c + im s) + i (im c - re s)
-          const float2 re = fma2(v.im, sn, mul2(v.re, c));
-          const float2 im = sub2(mul2(v.im, c), mul2(v.re, sn));
-          v.re = re;
-          v.im = im;
-        }
+        const cx& v = z[pos20(k1)];
         yrow[k1 * YROW] = make_float4(v.re.x, v.re.y, v.im.x, v.im.y);
       }
     }
@@ -826,6 +835,7 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
       if (a.mode == 0) setup_offline(N, a, nd, span);
       else setup_stream(N, a, next);
       if (N.tma) N.bar_parity = cur ? (armed0++) & 1 : (armed1++) & 1;
+      N.copy_ok = 1;
     }
     group_sync(grp);
 
