@@ -318,6 +318,14 @@ __device__ __forceinline__ int pcol(int f, int par) { return (2 * (f & 15) + (f 
 __device__ __forceinline__ void group_sync(int g) {
   asm volatile("bar.sync %0, %1;" ::"r"(g + 1), "r"(GROUP_THREADS) : "memory");
 }
+// A second barrier per tile group (ids 4..6) for one-way hand-offs: the
+// consumer warp waits, the producer warps only signal.
+__device__ __forceinline__ void group_wait2(int g) {
+  asm volatile("bar.sync %0, %1;" ::"r"(g + 1 + MAX_TILE_GROUPS), "r"(GROUP_THREADS) : "memory");
+}
+__device__ __forceinline__ void group_arrive2(int g) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(g + 1 + MAX_TILE_GROUPS), "r"(GROUP_THREADS) : "memory");
+}
 
 // Ampere-style asynchronous global -> shared copies (4 or 8 bytes, L1-allocating).
 __device__ __forceinline__ void cp_async4(float* dst, const float* src) {
@@ -920,8 +928,15 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
         mel_generic_warp(a, warp, PE, PO, orow);
       }
     }
-    if (a.bulk_store) fence_async_smem();   // the staged rows precede the bulk copies reading them
-    group_sync(grp);
+    if (a.bulk_store) {
+      // the staged rows precede the bulk copies reading them; only warp 0,
+      // which issues the copies, waits for every warp's rows
+      fence_async_smem();
+      if (warp == 0) group_wait2(grp);
+      else group_arrive2(grp);
+    } else {
+      group_sync(grp);   // every warp stores rows written by every warp
+    }
 
     // ---- store: the staged rows of the tile's frames ---------------------
     {
