@@ -278,6 +278,7 @@ struct __align__(16) Ctl {
   int copy_ok;              // verdict on the bulk copies (0: a thread's bounded wait gave up)
   int tmap_row;             // tensor row of the span's first sample (tma == 2)
   TileDesc pending;         // offline: the descriptor of the group's tile after next
+  int early;                // 1: the first tile's copy was issued before the prologue's barrier
 };
 constexpr int TAB_BYTES = (int)((sizeof(Tables) + 127) / 128 * 128);
 constexpr int CTL_BYTES = (int)((sizeof(Ctl) + 127) / 128 * 128);   // span region 128-byte aligned
@@ -308,6 +309,10 @@ static_assert(YBUF_BYTES % 128 == 0 && CTL_BYTES % 128 == 0 && TAB_BYTES % 128 =
 __host__ __device__ constexpr int group_bytes_for(int span_blocks, int n_mels) {
   return (2 * CTL_BYTES + ybuf_bytes_for(n_mels) + span_blocks * BLK * 4 + 127) / 128 * 128;
 }
+// Three offline tile groups of the default 128-band layout must fit in the
+// 232,448 bytes of shared memory an sm_100 CTA may opt into (15 warps per SM).
+static_assert(TAB_BYTES + MAX_TILE_GROUPS * group_bytes_for(OFFLINE_SPAN_BLOCKS, 128) <= 232448,
+              "three default tile groups per CTA");
 
 // Power-row column of frame slot f for a bin of parity par: the frames d and
 // d + 16 of a pair sit in columns 2d and 2d + 1, and odd bins swap the two
@@ -720,6 +725,34 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
   const int stride = gridDim.x * G;               // a group's tiles: first + k * stride
 
   Tables& tab = *reinterpret_cast<Tables*>(smem_raw);
+  unsigned char* gbase = smem_raw + TAB_BYTES + (size_t)grp * a.group_bytes;
+  Ctl* const ctl0 = reinterpret_cast<Ctl*>(gbase);
+  Ctl* const ctl1 = reinterpret_cast<Ctl*>(gbase + CTL_BYTES);
+  float4* const Y = reinterpret_cast<float4*>(gbase + 2 * CTL_BYTES);
+  float* const span = reinterpret_cast<float*>(gbase + 2 * CTL_BYTES + a.ybuf_bytes);
+  float* const Pbuf = reinterpret_cast<float*>(Y);   // power rows, after pass B has read Y
+  float* const orows = Pbuf + PROWS_FLOATS;          // staged output rows, after the power rows
+  const int opitch = orow_floats(a.n_mels);
+  int tile = blockIdx.x * G + grp;
+  int armed0 = 0, armed1 = 0;   // COPY_TID: bulk-copy uses of each control buffer
+
+  if (tid == COPY_TID) {
+    mbar_init(&ctl0->bar);
+    mbar_init(&ctl1->bar);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    // with the batch's index map in the parameters, the first tile's span
+    // copy (one tensor copy) can leave before the tables are staged
+    ctl0->early = 0;
+    if (tile < a.num_tiles && a.mode == 0 && a.meta_inline) {
+      setup_offline(*ctl0, a, inline_desc(a, tile), span);
+      if (ctl0->tma == 2) {
+        ctl0->bar_parity = (armed0++) & 1;
+        ctl0->copy_ok = 1;
+        ctl0->early = 1;
+        stage_tile(*ctl0, span, tid, a);
+      }
+    }
+  }
   {  // FFT tables -> shared memory, once per CTA
     const float4* src = reinterpret_cast<const float4*>(a.tables);
     float4* dst = reinterpret_cast<float4*>(smem_raw);
@@ -732,34 +765,19 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
       if (t < a.num_tiles) a.tiles[t] = offline_desc(a, t);
     }
   }
-  __syncthreads();
+  __syncthreads();   // tables, descriptors and the initialised mbarriers
 
-  unsigned char* gbase = smem_raw + TAB_BYTES + (size_t)grp * a.group_bytes;
-  Ctl* const ctl0 = reinterpret_cast<Ctl*>(gbase);
-  Ctl* const ctl1 = reinterpret_cast<Ctl*>(gbase + CTL_BYTES);
-  if (tid == COPY_TID) {
-    mbar_init(&ctl0->bar);
-    mbar_init(&ctl1->bar);
-    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-  }
-  int armed0 = 0, armed1 = 0;   // COPY_TID: bulk-copy uses of each control buffer
-  __syncthreads();
-  float4* const Y = reinterpret_cast<float4*>(gbase + 2 * CTL_BYTES);
-  float* const span = reinterpret_cast<float*>(gbase + 2 * CTL_BYTES + a.ybuf_bytes);
-  float* const Pbuf = reinterpret_cast<float*>(Y);   // power rows, after pass B has read Y
-  float* const orows = Pbuf + PROWS_FLOATS;          // staged output rows, after the power rows
-  const int opitch = orow_floats(a.n_mels);
-
-  int tile = blockIdx.x * G + grp;
   if (tile < a.num_tiles) {
-    if (tid == COPY_TID) {
-      if (a.mode == 0) setup_offline(*ctl0, a, tile_desc(a, tile), span);
-      else setup_stream(*ctl0, a, tile);
-      if (ctl0->tma) ctl0->bar_parity = (armed0++) & 1;
-      ctl0->copy_ok = 1;
+    if (!ctl0->early) {
+      if (tid == COPY_TID) {
+        if (a.mode == 0) setup_offline(*ctl0, a, tile_desc(a, tile), span);
+        else setup_stream(*ctl0, a, tile);
+        if (ctl0->tma) ctl0->bar_parity = (armed0++) & 1;
+        ctl0->copy_ok = 1;
+      }
+      group_sync(grp);
+      stage_tile(*ctl0, span, tid, a);
     }
-    group_sync(grp);
-    stage_tile(*ctl0, span, tid, a);
     if (tid == COPY_TID && a.mode == 0 && tile + stride < a.num_tiles) ctl0->pending = tile_desc(a, tile + stride);
   }
   int cur = 0;
