@@ -171,11 +171,12 @@ class Plan:
             _check(_lib.logmel_plan_create(sr, n_fft, hop, n_mels, fmin, fmax, ctypes.byref(h)),
                    "logmel_plan_create")
         self._h = h
+        self._destroy = _lib.logmel_plan_destroy   # kept: module globals may be gone at exit
 
     def __del__(self):
         h = getattr(self, "_h", None)
         if h is not None and h.value:
-            _lib.logmel_plan_destroy(h)
+            self._destroy(h)
             self._h = None
 
     def num_frames(self, n_samples: int) -> int:
@@ -229,11 +230,12 @@ class Stream:
         with torch.cuda.device(plan.device):
             _check(_lib.logmel_stream_create(plan._h, n_streams, ctypes.byref(h)), "logmel_stream_create")
         self._h = h
+        self._destroy = _lib.logmel_stream_destroy   # kept: module globals may be gone at exit
 
     def __del__(self):
         h = getattr(self, "_h", None)
         if h is not None and h.value:
-            _lib.logmel_stream_destroy(h)
+            self._destroy(h)
             self._h = None
 
     def frames_for_push(self, stream_id: int, length: int) -> int:
