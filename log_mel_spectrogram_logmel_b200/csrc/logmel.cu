@@ -113,6 +113,15 @@ int encode_out_map(CUtensorMap* m, float* out, int64_t rows, int n_mels) {
              : 0;
 }
 
+// True when some utterance with frames starts at an odd float offset from a
+// 16-byte boundary (every tile of an utterance shares its start's parity).
+bool has_odd_spans(const float* pcm, const int64_t* off, int64_t n_utt) {
+  const uint64_t base = reinterpret_cast<uintptr_t>(pcm) >> 2;
+  for (int64_t u = 0; u < n_utt; ++u)
+    if (frames_of(off[u + 1] - off[u]) > 0 && ((base + (uint64_t)off[u]) & 1)) return true;
+  return false;
+}
+
 }  // namespace
 
 struct LaunchCfg {
@@ -330,12 +339,14 @@ static void shape_launch(LaunchCfg& c, int span_blocks, int n_mels, int max_smem
 template <bool kDefault>
 static logmel_status setup_kernel(logmel_plan* p, int sms) {
   const size_t mx = std::max(p->off.smem, p->str.smem);
-  if (cudaFuncSetAttribute(logmel_fused_kernel<kDefault>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(logmel_fused_kernel<kDefault, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)mx) != cudaSuccess ||
+      cudaFuncSetAttribute(logmel_fused_kernel<kDefault, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)mx) != cudaSuccess)
     return LOGMEL_ERR_CUDA;
   for (LaunchCfg* c : {&p->off, &p->str}) {
     int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, logmel_fused_kernel<kDefault>,
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, logmel_fused_kernel<kDefault, false>,
                                                       c->groups * GROUP_THREADS, c->smem) != cudaSuccess ||
         occ < 1)
       return LOGMEL_ERR_CUDA;
@@ -344,7 +355,9 @@ static logmel_status setup_kernel(logmel_plan* p, int sms) {
   return LOGMEL_OK;
 }
 
-static cudaError_t launch(const logmel_plan* p, Args& a, int64_t tiles, cudaStream_t s) {
+// odd: some utterance of this offline batch starts at an odd float offset
+// from a 16-byte boundary (launch the kernel that can read such spans).
+static cudaError_t launch(const logmel_plan* p, Args& a, int64_t tiles, cudaStream_t s, bool odd = false) {
   const LaunchCfg& c = a.mode == 0 ? p->off : p->str;
   {
     const cudaError_t pending = cudaGetLastError();
@@ -365,10 +378,13 @@ static cudaError_t launch(const logmel_plan* p, Args& a, int64_t tiles, cudaStre
   std::memcpy(a.warp_band, p->mel.warp_band, sizeof a.warp_band);
   const int grid = (int)std::min<int64_t>((tiles + c.groups - 1) / c.groups, c.max_ctas);
   const int block = c.groups * GROUP_THREADS;
-  if (p->default_mel)
-    logmel_fused_kernel<true><<<grid, block, c.smem, s>>>(a);
-  else
-    logmel_fused_kernel<false><<<grid, block, c.smem, s>>>(a);
+  if (p->default_mel) {
+    if (odd) logmel_fused_kernel<true, true><<<grid, block, c.smem, s>>>(a);
+    else logmel_fused_kernel<true, false><<<grid, block, c.smem, s>>>(a);
+  } else {
+    if (odd) logmel_fused_kernel<false, true><<<grid, block, c.smem, s>>>(a);
+    else logmel_fused_kernel<false, false><<<grid, block, c.smem, s>>>(a);
+  }
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     char what[96];
@@ -621,8 +637,9 @@ logmel_status logmel_compute(logmel_plan* p, const float* pcm, const int64_t* of
   a.num_tiles = (int)tiles;
   a.n_mels = p->n_mels;
   a.pcm = pcm;
+  a.pcm_len = off[n_utt];
   a.n_utt = (int)n_utt;
-  if (launch(p, a, tiles, s) != cudaSuccess) return LOGMEL_ERR_CUDA;
+  if (launch(p, a, tiles, s, has_odd_spans(pcm, off, n_utt)) != cudaSuccess) return LOGMEL_ERR_CUDA;
   return LOGMEL_OK;
 }
 
@@ -1004,7 +1021,8 @@ extern "C" logmel_status logmel_compute_noalloc(const float* pcm, const int64_t*
   a.num_tiles = (int)tiles;
   a.n_mels = d.plan.n_mels;
   a.pcm = pcm;
+  a.pcm_len = off[n_utt];
   a.n_utt = (int)n_utt;
-  if (launch(&d.plan, a, tiles, s) != cudaSuccess) return LOGMEL_ERR_CUDA;
+  if (launch(&d.plan, a, tiles, s, has_odd_spans(pcm, off, n_utt)) != cudaSuccess) return LOGMEL_ERR_CUDA;
   return LOGMEL_OK;
 }

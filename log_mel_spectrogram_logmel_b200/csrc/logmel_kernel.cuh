@@ -128,6 +128,7 @@ struct Args {
   int n_mels;
   // offline
   const float* pcm;
+  int64_t pcm_len;             // samples in the PCM buffer (bounds the shifted block copies)
   const int64_t* sample_off;   // [n_utt + 1]
   const int64_t* frame_off;    // [n_utt + 1]
   const int* tile_off;         // [n_utt + 1]
@@ -248,6 +249,30 @@ __device__ __forceinline__ void dft10(cx (&x)[10]) {
          x[(5 * k1 + 8) % 10]);
 }
 
+// Pass A input: z[m1] = windowed (x[n], x[n + 1]) of the pair's two frames,
+// n = 20 m1 + 2 m2, read from the staged span (kOdd: the samples sit at an
+// odd float offset, so each pair takes two 4-byte loads).
+template <bool kOdd>
+__device__ __forceinline__ void window_load(cx (&z)[N1], const float* sa, const float* sb, const Tables& tab,
+                                            int m2) {
+#pragma unroll
+  for (int m1 = 0; m1 < N1; ++m1) {
+    const int off = BLK * (m1 / 8) + 20 * (m1 % 8);   // sample n = 20 m1 + 2 m2
+    float2 xa, xb;
+    if constexpr (kOdd) {
+      xa = make_float2(sa[off], sa[off + 1]);
+      xb = make_float2(sb[off], sb[off + 1]);
+    } else {
+      xa = *reinterpret_cast<const float2*>(sa + off);
+      xb = *reinterpret_cast<const float2*>(sb + off);
+    }
+    const float4 w4 = *reinterpret_cast<const float4*>(&tab.win[m2][m1 & ~1]);
+    const float2 w = (m1 & 1) ? make_float2(w4.z, w4.w) : make_float2(w4.x, w4.y);
+    z[m1].re = make_float2(xa.x * w.x, xb.x * w.x);
+    z[m1].im = make_float2(xa.y * w.y, xb.y * w.y);
+  }
+}
+
 __device__ __forceinline__ cx sel(bool p, const cx& a, const cx& b) {
   return p ? a : b;
 }
@@ -273,7 +298,9 @@ struct __align__(16) Ctl {
   unsigned long long bar;   // mbarrier completing this buffer's bulk span copies
   int ngroups;
   int nslots;
-  int tma;                  // 1: per-block bulk copies, 2: one tensor copy (wait on bar)
+  int tma;                  // 1: per-block bulk copies, 2: one tensor copy, 3..5: per-block
+                            // bulk copies from 16-byte boundaries, samples shifted by tma - 2
+                            // within each slot (all wait on bar); 0: cp.async
   int bar_parity;           // phase of bar to wait for
   int copy_ok;              // verdict on the bulk copies (0: a thread's bounded wait gave up)
   int tmap_row;             // tensor row of the span's first sample (tma == 2)
@@ -464,7 +491,8 @@ __device__ __forceinline__ TileDesc tile_desc(const Args& a, int t) {
   return a.meta_inline ? inline_desc(a, t) : a.tiles[t];
 }
 
-__device__ void setup_offline(Ctl& S, const Args& a, const TileDesc& t, const float* span) {
+// odd_ok: the kernel can read spans staged at an odd float offset.
+__device__ void setup_offline(Ctl& S, const Args& a, const TileDesc& t, const float* span, bool odd_ok) {
   Group& g = S.groups[0];
   g.src0 = a.pcm + t.src;
   g.src1 = nullptr;
@@ -483,11 +511,19 @@ __device__ void setup_offline(Ctl& S, const Args& a, const TileDesc& t, const fl
   // source is 16-byte aligned; else cp.async
   const int64_t row = t.src / HOP;
   const int nb = (g.nstage + HOP - 1) / HOP;
+  const int r = (int)((reinterpret_cast<uintptr_t>(g.src0) >> 2) & 3);   // floats past a 16-byte boundary
   if (a.tmap_rows > 0 && t.src % HOP == 0 && row + nb <= a.tmap_rows && (smem_addr(span) & 127) == 0) {
     S.tma = 2;
     S.tmap_row = (int)row;
+  } else if ((reinterpret_cast<uintptr_t>(g.src0) & 15) == 0) {
+    S.tma = 1;
+  } else if ((odd_ok || !(r & 1)) && (reinterpret_cast<uintptr_t>(g.src0) & 3) == 0 && g.src0 - r >= a.pcm &&
+             g.src0 - r + ((g.nstage + r + 3) & ~3) <= a.pcm + a.pcm_len) {
+    // each hop block from the 16-byte boundary at or before it: its slot then
+    // holds the block's 160 samples from position r (r + 159 < 164)
+    S.tma = 2 + r;
   } else {
-    S.tma = (reinterpret_cast<uintptr_t>(g.src0) & 15) == 0;
+    S.tma = 0;
   }
 }
 
@@ -550,6 +586,22 @@ __device__ __forceinline__ void stage_tile(Ctl& S, float* span, int tid, const A
     if (tid == COPY_TID) {
       mbar_expect_tx(&S.bar, (unsigned)(BLK * OFFLINE_SPAN_BLOCKS * 4));
       tensor_load_2d(span, &a.tmap, 0, S.tmap_row, &S.bar);
+    }
+    return;
+  }
+  if (S.tma >= 3) {   // shifted: 164 floats per hop block from the 16-byte boundary before it
+    const Group& g = S.groups[0];
+    if (tid >= COPY_TID && tid < COPY_TID + 32) {
+      const int l = tid - COPY_TID;
+      const int r = S.tma - 2;
+      const int nb = (g.nstage + HOP - 1) / HOP;
+      const int total = (g.nstage + r + 3) & ~3;   // floats from src0 - r, a multiple of 4
+      if (l == 0) mbar_expect_tx(&S.bar, 4u * (unsigned)(BLK * (nb - 1) + (total - HOP * (nb - 1))));
+      __syncwarp();
+      for (int b = l; b < nb; b += 32) {
+        const int len = min(BLK, total - b * HOP);   // 164, the last block what is left
+        bulk_load(span + b * BLK, g.src0 - r + b * HOP, (unsigned)len * 4u, &S.bar);
+      }
     }
     return;
   }
@@ -711,7 +763,52 @@ __device__ __forceinline__ void split_power(const Tables& tab, const cx& zk, con
   pm = fma2(qi, qi, mul2(qr, qr));
 }
 
-template <bool kDefaultMel>
+// Pass A for one thread (frame pair d, role m2): windowed loads, 20-point
+// DFT over m1, twiddle; then, once the previous tile has released the pass
+// buffer (warp 0 waits for its row copies; group barrier), the stores of
+// the 20 outputs.  Returns the group's copy verdict (false: stop).
+template <bool kOdd>
+__device__ __forceinline__ bool pass_a(const Tables& tab, const float* span, const Ctl& S, float4* Y, int d,
+                                       int m2, int warp, int grp) {
+  const int sh = S.tma >= 3 ? S.tma - 2 : 0;
+  const float* sa = span + BLK * slot_block(S, d) + 2 * m2 + sh;
+  const float* sb = span + BLK * slot_block(S, d + DUOS) + 2 * m2 + sh;
+  cx z[N1];
+  window_load<kOdd>(z, sa, sb, tab, m2);
+  dft20(z);
+#pragma unroll
+  for (int k1 = 1; k1 < N1; ++k1) {
+    cx& v = z[pos20(k1)];
+    const float4 t = tab.w400[2 * m2 * k1];   // e^{-2 pi i m2 k1 / 200} = c - i s
+    const float2 c = make_float2(t.x, t.y), sn = make_float2(t.z, t.w);
+    // (re + i im)(c - i s) = (re c + im s) + i (im c - re s)
+    const float2 re = fma2(v.im, sn, mul2(v.re, c));
+    const float2 im = sub2(mul2(v.im, c), mul2(v.re, sn));
+    v.re = re;
+    v.im = im;
+  }
+  // the previous tile's mel stage and row copies are done with the pass
+  // buffer before it is overwritten, and every copy verdict is in
+  if (warp == 0) bulk_wait_read();
+  group_sync(grp);
+  if (!S.copy_ok) return false;
+  float4* yrow = Y + d * YDUO + m2;
+#pragma unroll
+  for (int k1 = 0; k1 < N1; ++k1) {
+    const cx& v = z[pos20(k1)];
+    yrow[k1 * YROW] = make_float4(v.re.x, v.re.y, v.im.x, v.im.y);
+  }
+  return true;
+}
+__device__ __noinline__ bool pass_a_odd(const Tables& tab, const float* span, const Ctl& S, float4* Y, int d,
+                                        int m2, int warp, int grp) {
+  return pass_a<true>(tab, span, S, Y, d, m2, warp, grp);
+}
+
+// kOddSpans: offline batches in which some utterance starts at an odd float
+// offset from a 16-byte boundary; such spans are read by an out-of-line copy
+// of pass A (elsewhere they fall back to cp.async staging).
+template <bool kDefaultMel, bool kOddSpans>
 __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fused_kernel(const __grid_constant__ Args a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   const int G = blockDim.x / GROUP_THREADS;
@@ -744,7 +841,7 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
     // copy (one tensor copy) can leave before the tables are staged
     ctl0->early = 0;
     if (tile < a.num_tiles && a.mode == 0 && a.meta_inline) {
-      setup_offline(*ctl0, a, inline_desc(a, tile), span);
+      setup_offline(*ctl0, a, inline_desc(a, tile), span, kOddSpans);
       if (ctl0->tma == 2) {
         ctl0->bar_parity = (armed0++) & 1;
         ctl0->copy_ok = 1;
@@ -770,7 +867,7 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
   if (tile < a.num_tiles) {
     if (!ctl0->early) {
       if (tid == COPY_TID) {
-        if (a.mode == 0) setup_offline(*ctl0, a, tile_desc(a, tile), span);
+        if (a.mode == 0) setup_offline(*ctl0, a, tile_desc(a, tile), span, kOddSpans);
         else setup_stream(*ctl0, a, tile);
         if (ctl0->tma) ctl0->bar_parity = (armed0++) & 1;
         ctl0->copy_ok = 1;
@@ -815,50 +912,23 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
     }
 
     // ---- pass A: window, 20-point DFTs over m1, twiddle --------------------
+    // (spans staged at an odd float offset take a separate, out-of-line copy
+    // of the pass, so that the common path keeps its register allocation)
     {
-      const int m2 = role;
-      const float* sa = span + BLK * slot_block(S, d) + 2 * m2;
-      const float* sb = span + BLK * slot_block(S, d + DUOS) + 2 * m2;
-      cx z[N1];
-#pragma unroll
-      for (int m1 = 0; m1 < N1; ++m1) {
-        const int off = BLK * (m1 / 8) + 20 * (m1 % 8);   // sample n = 20 m1 + 2 m2
-        const float2 xa = *reinterpret_cast<const float2*>(sa + off);
-        const float2 xb = *reinterpret_cast<const float2*>(sb + off);
-        const float4 w4 = *reinterpret_cast<const float4*>(&tab.win[m2][m1 & ~1]);
-        const float2 w = (m1 & 1) ? make_float2(w4.z, w4.w) : make_float2(w4.x, w4.y);
-        z[m1].re = make_float2(xa.x * w.x, xb.x * w.x);
-        z[m1].im = make_float2(xa.y * w.y, xb.y * w.y);
-      }
-      dft20(z);
-#pragma unroll
-      for (int k1 = 1; k1 < N1; ++k1) {
-        cx& v = z[pos20(k1)];
-        const float4 t = tab.w400[2 * m2 * k1];   // e^{-2 pi i m2 k1 / 200} = c - i s
-        const float2 c = make_float2(t.x, t.y), sn = make_float2(t.z, t.w);
-        // (re + i im)(c - i s) = (re c + im s) + i (im c - re s)
-        const float2 re = fma2(v.im, sn, mul2(v.re, c));
-        const float2 im = sub2(mul2(v.im, c), mul2(v.re, sn));
-        v.re = re;
-        v.im = im;
-      }
-      // the previous tile's mel stage and row copies are done with the pass
-      // buffer before it is overwritten, and every copy verdict is in
-      if (warp == 0) bulk_wait_read();
-      group_sync(grp);
-      if (!S.copy_ok) {   // a bulk copy never completed: flag it and stop this group
+      const int sh = S.tma >= 3 ? S.tma - 2 : 0;   // shifted block copies: samples start at sh
+      bool ok;
+      if constexpr (kOddSpans)
+        ok = (sh & 1) ? pass_a_odd(tab, span, S, Y, d, role, warp, grp)
+                      : pass_a<false>(tab, span, S, Y, d, role, warp, grp);
+      else
+        ok = pass_a<false>(tab, span, S, Y, d, role, warp, grp);
+      if (!ok) {   // a bulk copy never completed: flag it and stop this group
         if (tid == COPY_TID) atomicExch(a.status, STATUS_COPY_TIMEOUT);
         break;
       }
-      float4* yrow = Y + d * YDUO + m2;
-#pragma unroll
-      for (int k1 = 0; k1 < N1; ++k1) {
-        const cx& v = z[pos20(k1)];
-        yrow[k1 * YROW] = make_float4(v.re.x, v.re.y, v.im.x, v.im.y);
-      }
     }
     if (tid == COPY_TID && next < a.num_tiles) {   // the next tile's groups
-      if (a.mode == 0) setup_offline(N, a, nd, span);
+      if (a.mode == 0) setup_offline(N, a, nd, span, kOddSpans);
       else setup_stream(N, a, next);
       if (N.tma) N.bar_parity = cur ? (armed0++) & 1 : (armed1++) & 1;
       N.copy_ok = 1;
