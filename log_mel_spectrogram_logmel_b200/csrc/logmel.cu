@@ -93,6 +93,46 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
+// The PCM as a 3-D tensor [rows][40][w] whose element (x, y, z) is
+// pcm[160 z + 4 y + x]: rows of w samples start at every 16-byte boundary
+// (for w = 164 the strides overlap on purpose), so one 164 x 1 x 34 box
+// lands any tile's span, from the boundary at or before it, in its
+// hop-block slots.  Rows are counted so that every row of every start class
+// lies inside the first `total` samples.  Returns the rows, or 0 when no
+// map can be made.
+int encode_pcm_map(CUtensorMap* m, const float* pcm, int64_t total, int w = BLK) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  const int64_t rows = total >= 4 * (HOP / 4 - 1) + w ? (total - 4 * (HOP / 4 - 1) - w) / HOP + 1 : 0;
+  if (!enc || (reinterpret_cast<uintptr_t>(pcm) & 15) || rows < 1 || rows >= INT32_MAX) return 0;
+  cuuint64_t dims[3] = {(cuuint64_t)w, (cuuint64_t)(HOP / 4), (cuuint64_t)rows};
+  cuuint64_t strides[2] = {4 * sizeof(float), (cuuint64_t)HOP * sizeof(float)};
+  cuuint32_t box[3] = {(cuuint32_t)BLK, 1, (cuuint32_t)OFFLINE_SPAN_BLOCKS};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(pcm), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS
+             ? (int)rows
+             : 0;
+}
+
+// The PCM as a 2-D tensor of 160-sample rows (contiguous) for one-box copies
+// of spans that start on a row; the box is 164 x 34 and its columns
+// 160..163 lie outside the tensor (zeros).  Returns the rows, or 0.
+int encode_pcm_rows(CUtensorMap* m, const float* pcm, int64_t total) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  const int64_t rows = total / HOP;
+  if (!enc || (reinterpret_cast<uintptr_t>(pcm) & 15) || rows < 1 || rows >= INT32_MAX) return 0;
+  cuuint64_t dims[2] = {(cuuint64_t)HOP, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)HOP * sizeof(float)};
+  cuuint32_t box[2] = {(cuuint32_t)BLK, (cuuint32_t)OFFLINE_SPAN_BLOCKS};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(pcm), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS
+             ? (int)rows
+             : 0;
+}
+
 // The output rows as a 2-D tensor [rows][n_mels] for one-box stores of full
 // tiles: the box is orow_floats(n_mels) x 32, matching the staged rows in
 // shared memory; its pad columns lie outside the tensor and are not written.
@@ -150,10 +190,10 @@ struct logmel_plan {
   Args mel{};               // filterbank fields copied into every launch
   bool default_mel = false; // structure equals the compiled default layout
   // tensor map of the last offline PCM buffer (re-encoded when it changes)
-  CUtensorMap tmap{};
+  CUtensorMap tmap{}, tmap_s{};
   const float* tmap_pcm = nullptr;
   int64_t tmap_len = -1;
-  int tmap_rows = 0;
+  int tmap_rows = 0, tmap_s_rows = 0;
   // tensor map of the last offline output buffer (full-tile row stores)
   CUtensorMap otmap{};
   const float* otmap_out = nullptr;
@@ -602,29 +642,19 @@ logmel_status logmel_compute(logmel_plan* p, const float* pcm, const int64_t* of
   a.out = out;
   a.status = p->d_status;
   a.mode = 0;
-  // the PCM as rows of 160 samples for one-box tile copies (16-byte aligned
-  // base and at least one full row); the box is 164 x 34: columns 160..163
-  // are outside the tensor and arrive as zeros
+  // the PCM as a tensor for one-box tile copies (re-encoded when the buffer
+  // or its length changes)
   const int64_t total = off[n_utt];
   if (pcm != p->tmap_pcm || total != p->tmap_len) {
     p->tmap_pcm = pcm;
     p->tmap_len = total;
-    p->tmap_rows = 0;
-    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
-    const int64_t rows = total / HOP;
-    if (enc && (reinterpret_cast<uintptr_t>(pcm) & 15) == 0 && rows >= 1 && rows < INT32_MAX) {
-      cuuint64_t dims[2] = {(cuuint64_t)HOP, (cuuint64_t)rows};
-      cuuint64_t strides[1] = {(cuuint64_t)HOP * sizeof(float)};
-      cuuint32_t box[2] = {(cuuint32_t)BLK, (cuuint32_t)OFFLINE_SPAN_BLOCKS};
-      cuuint32_t estr[2] = {1, 1};
-      if (enc(&p->tmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(pcm), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
-        p->tmap_rows = (int)rows;
-    }
+    p->tmap_rows = encode_pcm_rows(&p->tmap, pcm, total);
+    p->tmap_s_rows = encode_pcm_map(&p->tmap_s, pcm, total, BLK);
   }
   a.tmap = p->tmap;
   a.tmap_rows = p->tmap_rows;
+  a.tmap_s = p->tmap_s;
+  a.tmap_s_rows = p->tmap_s_rows;
   if (p->default_mel) {
     if (out != p->otmap_out || frames != p->otmap_len) {
       p->otmap_out = out;
@@ -1002,21 +1032,9 @@ extern "C" logmel_status logmel_compute_noalloc(const float* pcm, const int64_t*
   a.out = out;
   a.status = status;
   a.mode = 0;
-  // the PCM as rows of 160 samples for one-box tile copies, as in logmel_compute
-  const int64_t total = off[n_utt];
-  const int64_t rows = total / HOP;
-  a.tmap_rows = 0;
-  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
-  if (enc && (reinterpret_cast<uintptr_t>(pcm) & 15) == 0 && rows >= 1 && rows < INT32_MAX) {
-    cuuint64_t dims[2] = {(cuuint64_t)HOP, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)HOP * sizeof(float)};
-    cuuint32_t box[2] = {(cuuint32_t)BLK, (cuuint32_t)OFFLINE_SPAN_BLOCKS};
-    cuuint32_t estr[2] = {1, 1};
-    if (enc(&a.tmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(pcm), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
-      a.tmap_rows = (int)rows;
-  }
+  // the PCM as a tensor for one-box tile copies, as in logmel_compute
+  a.tmap_rows = encode_pcm_rows(&a.tmap, pcm, off[n_utt]);
+  a.tmap_s_rows = encode_pcm_map(&a.tmap_s, pcm, off[n_utt], BLK);
   a.otmap_rows = encode_out_map(&a.otmap, out, frames, d.plan.n_mels);
   a.num_tiles = (int)tiles;
   a.n_mels = d.plan.n_mels;

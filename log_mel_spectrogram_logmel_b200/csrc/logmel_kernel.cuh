@@ -104,17 +104,23 @@ struct TileDesc {
 };
 
 struct Args {
-  // offline: the PCM as a 2-D tensor of 160-sample rows; a 164 x 34 box
-  // lands one tile's span in its hop-block slots (columns 160..163 of a box
-  // row are outside the tensor and read as zeros: padding)
+  // offline: two tensor views of the PCM for one-box tile copies.
+  // tmap: rows of 160 samples (2-D, contiguous rows); a 164 x 34 box lands a
+  // span that starts on a row in its hop-block slots, columns 160..163 lying
+  // outside the tensor (zeros, not read).  tmap_s: a 3-D tensor whose
+  // element (x, y, z) is pcm[160 z + 4 y + x], rows of 164 samples starting
+  // at every 16-byte boundary (overlapping strides); a 164 x 1 x 34 box lands
+  // any other span from the boundary at or before it, shifted by its offset.
   CUtensorMap tmap;
+  CUtensorMap tmap_s;
   // offline: the output as a 2-D tensor [rows][n_mels]; an
   // orow_floats(n_mels) x 32 box stores one full tile's staged rows (the pad
   // columns fall outside the tensor)
   CUtensorMap otmap;
-  int tmap_rows;        // rows of the input tensor (0: no tensor map)
+  int tmap_rows;        // rows of tmap (0: no tensor map)
+  int tmap_s_rows;      // rows (z extent) of tmap_s (0: none)
   int otmap_rows;       // rows of the output tensor (0: no tensor map)
-  int pad_tm_[2];
+  int pad_tm_[1];
   const Tables* tables;
   TileDesc* tiles;      // offline: per-tile descriptors (written by the kernel's prologue)
   float* out;
@@ -298,12 +304,14 @@ struct __align__(16) Ctl {
   unsigned long long bar;   // mbarrier completing this buffer's bulk span copies
   int ngroups;
   int nslots;
-  int tma;                  // 1: per-block bulk copies, 2: one tensor copy, 3..5: per-block
-                            // bulk copies from 16-byte boundaries, samples shifted by tma - 2
-                            // within each slot (all wait on bar); 0: cp.async
+  int tma;                  // staging: kind | (shift << 2).  kind 0: cp.async; 1: bulk copies
+                            // per hop block; 2: one tensor copy (both wait on bar).  shift
+                            // (0..3): the slots hold their samples from position shift
+                            // (copies start at the 16-byte boundary before the span)
   int bar_parity;           // phase of bar to wait for
   int copy_ok;              // verdict on the bulk copies (0: a thread's bounded wait gave up)
-  int tmap_row;             // tensor row of the span's first sample (tma == 2)
+  int tmap_row;             // tensor copy: row and start class of the box (see Args::tmap)
+  int tmap_y;
   TileDesc pending;         // offline: the descriptor of the group's tile after next
   int early;                // 1: the first tile's copy was issued before the prologue's barrier
 };
@@ -403,6 +411,14 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, unsigned b
                    smem_addr(dst)),
                "l"(src), "r"(bytes), "r"(smem_addr(bar))
                : "memory");
+}
+__device__ __forceinline__ void tensor_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z,
+                                               unsigned long long* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];\n" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
+      : "memory");
 }
 __device__ __forceinline__ void tensor_load_2d(void* dst, const CUtensorMap* map, int x, int y,
                                                unsigned long long* bar) {
@@ -506,22 +522,28 @@ __device__ void setup_offline(Ctl& S, const Args& a, const TileDesc& t, const fl
   g.carry_len_dst = nullptr;
   S.ngroups = 1;
   S.nslots = t.nframes;
-  // one tensor copy when the span starts on a tensor row and its last hop
-  // block is a whole row of the tensor; else per-block bulk copies when the
-  // source is 16-byte aligned; else cp.async
-  const int64_t row = t.src / HOP;
+  // Staging from the 16-byte boundary at or before the span (r floats
+  // earlier): every slot then holds its hop block's 160 samples from position
+  // r (r + 159 < 164).  One tensor copy when the map covers the span's rows;
+  // else one bulk copy per hop block; else cp.async.  Spans at an odd float
+  // offset need a kernel that reads them (odd_ok).
   const int nb = (g.nstage + HOP - 1) / HOP;
   const int r = (int)((reinterpret_cast<uintptr_t>(g.src0) >> 2) & 3);   // floats past a 16-byte boundary
-  if (a.tmap_rows > 0 && t.src % HOP == 0 && row + nb <= a.tmap_rows && (smem_addr(span) & 127) == 0) {
-    S.tma = 2;
+  const int64_t a0 = t.src - r;   // the map's base is 16-byte aligned: a0 is a multiple of 4
+  const int64_t row = a0 / HOP;
+  const bool shift_ok = odd_ok || !(r & 1);
+  const int yk = (int)(a0 - row * HOP) / 4;   // start class: 4 yk floats into a 160-sample row
+  const bool on_row = r == 0 && yk == 0;
+  const int map_rows = on_row ? a.tmap_rows : a.tmap_s_rows;
+  if (map_rows > 0 && shift_ok && a0 >= 0 && row + nb <= map_rows && (smem_addr(span) & 127) == 0) {
+    S.tma = 2 | (r << 2);
     S.tmap_row = (int)row;
+    S.tmap_y = on_row ? -1 : yk;   // -1: the 2-D row map
   } else if ((reinterpret_cast<uintptr_t>(g.src0) & 15) == 0) {
     S.tma = 1;
-  } else if ((odd_ok || !(r & 1)) && (reinterpret_cast<uintptr_t>(g.src0) & 3) == 0 && g.src0 - r >= a.pcm &&
+  } else if (shift_ok && (reinterpret_cast<uintptr_t>(g.src0) & 3) == 0 && g.src0 - r >= a.pcm &&
              g.src0 - r + ((g.nstage + r + 3) & ~3) <= a.pcm + a.pcm_len) {
-    // each hop block from the 16-byte boundary at or before it: its slot then
-    // holds the block's 160 samples from position r (r + 159 < 164)
-    S.tma = 2 + r;
+    S.tma = 1 | (r << 2);
   } else {
     S.tma = 0;
   }
@@ -582,18 +604,19 @@ __device__ void setup_stream(Ctl& S, const Args& a, int tile) {
 constexpr int COPY_TID = 128;
 
 __device__ __forceinline__ void stage_tile(Ctl& S, float* span, int tid, const Args& a) {
-  if (S.tma == 2) {   // one 164 x 34 tensor box per tile
+  if ((S.tma & 3) == 2) {   // one 164 x 1 x 34 tensor box per tile
     if (tid == COPY_TID) {
       mbar_expect_tx(&S.bar, (unsigned)(BLK * OFFLINE_SPAN_BLOCKS * 4));
-      tensor_load_2d(span, &a.tmap, 0, S.tmap_row, &S.bar);
+      if (S.tmap_y < 0) tensor_load_2d(span, &a.tmap, 0, S.tmap_row, &S.bar);
+      else tensor_load_3d(span, &a.tmap_s, 0, S.tmap_y, S.tmap_row, &S.bar);
     }
     return;
   }
-  if (S.tma >= 3) {   // shifted: 164 floats per hop block from the 16-byte boundary before it
+  if (S.tma >= 4) {   // shifted: 164 floats per hop block from the 16-byte boundary before it
     const Group& g = S.groups[0];
     if (tid >= COPY_TID && tid < COPY_TID + 32) {
       const int l = tid - COPY_TID;
-      const int r = S.tma - 2;
+      const int r = S.tma >> 2;
       const int nb = (g.nstage + HOP - 1) / HOP;
       const int total = (g.nstage + r + 3) & ~3;   // floats from src0 - r, a multiple of 4
       if (l == 0) mbar_expect_tx(&S.bar, 4u * (unsigned)(BLK * (nb - 1) + (total - HOP * (nb - 1))));
@@ -770,7 +793,7 @@ __device__ __forceinline__ void split_power(const Tables& tab, const cx& zk, con
 template <bool kOdd>
 __device__ __forceinline__ bool pass_a(const Tables& tab, const float* span, const Ctl& S, float4* Y, int d,
                                        int m2, int warp, int grp) {
-  const int sh = S.tma >= 3 ? S.tma - 2 : 0;
+  const int sh = S.tma >> 2;
   const float* sa = span + BLK * slot_block(S, d) + 2 * m2 + sh;
   const float* sb = span + BLK * slot_block(S, d + DUOS) + 2 * m2 + sh;
   cx z[N1];
@@ -842,7 +865,7 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
     ctl0->early = 0;
     if (tile < a.num_tiles && a.mode == 0 && a.meta_inline) {
       setup_offline(*ctl0, a, inline_desc(a, tile), span, kOddSpans);
-      if (ctl0->tma == 2) {
+      if ((ctl0->tma & 3) == 2) {
         ctl0->bar_parity = (armed0++) & 1;
         ctl0->copy_ok = 1;
         ctl0->early = 1;
@@ -915,7 +938,7 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
     // (spans staged at an odd float offset take a separate, out-of-line copy
     // of the pass, so that the common path keeps its register allocation)
     {
-      const int sh = S.tma >= 3 ? S.tma - 2 : 0;   // shifted block copies: samples start at sh
+      const int sh = S.tma >> 2;   // the slots hold their samples from position sh
       bool ok;
       if constexpr (kOddSpans)
         ok = (sh & 1) ? pass_a_odd(tab, span, S, Y, d, role, warp, grp)
