@@ -127,6 +127,29 @@ def test_edge_lengths_and_unaligned_offsets(plan):
     check_against_oracle(g, L, M)
 
 
+@pytest.mark.parametrize("base_shift", [0, 1, 2, 3])
+def test_span_staging_at_every_alignment(plan, base_shift):
+    """Utterances whose starts cover every residue mod 4 and several mod 160,
+    in a buffer that ends at the last utterance, with the buffer itself
+    starting 0..3 floats past a 16-byte boundary.  Tiles are staged by the
+    row tensor copy, the shifted tensor copy, per-block bulk copies (shifted
+    or not) or cp.async, depending on where they start and how close they
+    end to the buffer's end; every route must give the oracle's values."""
+    lengths = [16000 + 160 * 3, 4001, 16002, 8003, 12004, 160 * 50 + 1, 400, 20397, 9000 + 157, 5001, 402]
+    pcm_np, off = W.ragged_batch(lengths=lengths, seed0=7100)
+    starts = off[:-1] + base_shift
+    assert {int(v % 4) for v in starts} == {0, 1, 2, 3}
+    big = torch.zeros(len(pcm_np) + 8, dtype=torch.float32, device="cuda")
+    pcm = big[base_shift:base_shift + len(pcm_np)]
+    pcm.copy_(torch.from_numpy(pcm_np).cuda())
+    assert pcm.is_contiguous() and (pcm.data_ptr() - big.data_ptr()) == 4 * base_shift
+    g = plan.compute(pcm, off)
+    torch.cuda.synchronize()
+    L, M = O.log_mel_batch(pcm_np, off, return_energy=True)
+    check_against_oracle(g.cpu().numpy(), L, M)
+    assert plan.device_status() == 0
+
+
 def test_zero_input_is_exact_floor(plan):
     g = _run(plan, np.zeros(48000, np.float32), [0, 48000])
     assert g.shape == (298, 128) and np.all(g == FLOOR32)
