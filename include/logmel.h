@@ -204,6 +204,66 @@ logmel_status logmel_stream_reset(logmel_stream* st, int stream_id, void* stream
 logmel_status logmel_compute_noalloc(const float* pcm, const int64_t* offsets, int64_t n_utt,
                                      float* out, int* device_status, void* stream);
 
+/* ---- Encoder-ready index maps over the log-mel rows (host only) ----------
+ * The steps right after the log-mel front-end cut its rows into encoder
+ * inputs.  These calls only compute row ranges: the encoder takes views of
+ * the rows logmel_compute (or a stream's pushes) wrote; nothing is copied. */
+
+/* One offline encoder chunk: rows [row, row + frames) of the output,
+ * belonging to utterance utt, fed to the encoder padded to `padded` rows. */
+typedef struct {
+  int64_t utt;
+  int64_t row;
+  int64_t frames;
+  int64_t padded;
+} logmel_chunk;
+
+/* Offline chunks: "从零理解 ASR：音频基础、Qwen3-ASR 架构，以及离线 vs 流式推理原理",
+ * section 2.3 (preprocessor config chunk_length = 30 s = 3000 frames), and
+ * "Qwen3-ASR详解transcribe.cpp中audio-LLM token注入架构原理", section
+ * "4. Padding 浪费" (the encoder pads every input to 3000 frames; length
+ * buckets reduce the waste).  Utterance u's rows frame_offsets[u] ..
+ * frame_offsets[u + 1] (host, n_utt + 1 entries, as logmel_frame_offsets
+ * returns them) are cut into consecutive chunks of at most chunk_frames rows
+ * (3000); each is padded up to a multiple of quantum rows, at most
+ * chunk_frames (quantum = chunk_frames: pad every chunk to 3000; smaller:
+ * buckets).  Utterances without rows give no chunks.
+ *   logmel_encoder_chunk_count: the number of chunks, or -1 on a bad
+ *     argument (NULL offsets, n_utt < 0, chunk_frames < 1, decreasing offsets).
+ *   logmel_encoder_chunks: writes them in utterance order into chunks (host,
+ *     capacity entries).  *n_chunks (host) always receives the count; if it
+ *     exceeds capacity, or an argument is bad (also quantum < 1), nothing is
+ *     written and LOGMEL_ERR_INVALID_ARG is returned. */
+int64_t logmel_encoder_chunk_count(const int64_t* frame_offsets, int64_t n_utt, int64_t chunk_frames);
+logmel_status logmel_encoder_chunks(const int64_t* frame_offsets, int64_t n_utt, int64_t chunk_frames,
+                                    int64_t quantum, logmel_chunk* chunks, int64_t capacity, int64_t* n_chunks);
+
+/* One streaming encoder window: the encoder processes frames
+ * [ctx_begin, ctx_end) of the stream and keeps the results of its core
+ * frames [core_begin, core_end) (frame indices count the stream's frames
+ * from its first push). */
+typedef struct {
+  int64_t chunk;
+  int64_t core_begin;
+  int64_t core_end;
+  int64_t ctx_begin;
+  int64_t ctx_end;
+} logmel_window;
+
+/* Streaming windows: the first page, section 5.2 ("流式模式的滑动窗口机制"):
+ * chunk k covers frames [k * chunk_frames, (k + 1) * chunk_frames) (500) and
+ * is processed with `context` frames (n_window = 50) on each side, clipped at
+ * frame 0.  For a stream that has emitted n_frames frames, the windows are
+ * those whose right context has arrived ((k + 1) * chunk_frames + context <=
+ * n_frames); once the stream has finished (finished != 0), every chunk that
+ * holds a frame, with its core and context clipped at n_frames.  Writes them
+ * in order into windows (host, capacity entries); *n_windows (host) always
+ * receives the count; if it exceeds capacity, or n_frames < 0,
+ * chunk_frames < 1 or context < 0, nothing is written and
+ * LOGMEL_ERR_INVALID_ARG is returned. */
+logmel_status logmel_stream_windows(int64_t n_frames, int finished, int64_t chunk_frames, int64_t context,
+                                    logmel_window* windows, int64_t capacity, int64_t* n_windows);
+
 /* Reads and clears the plan's device status word (synchronises `stream`).
  * *code = 0 when no kernel has flagged an inconsistency since the last read. */
 logmel_status logmel_plan_device_status(logmel_plan* plan, int* code, void* stream);

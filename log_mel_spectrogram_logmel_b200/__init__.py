@@ -19,7 +19,8 @@ import os
 
 import numpy as np
 
-__all__ = ["Plan", "Stream", "LogMelError", "compute_noalloc", "lib_path", "exported_symbols", "STATUS"]
+__all__ = ["Plan", "Stream", "LogMelError", "compute_noalloc", "encoder_chunks", "stream_windows", "chunk_views",
+           "lib_path", "exported_symbols", "STATUS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "liblogmel_b200.so")
@@ -71,6 +72,9 @@ _SIGS = {
     "logmel_stream_set_state": (_i, [_p, _vp, _i64, _vp]),
     "logmel_stream_reset": (_i, [_p, _i, _vp]),
     "logmel_plan_device_status": (_i, [_p, ctypes.POINTER(_i), _vp]),
+    "logmel_encoder_chunk_count": (_i64, [_i64p, _i64, _i64]),
+    "logmel_encoder_chunks": (_i, [_i64p, _i64, _i64, _i64, _vp, _i64, _i64p]),
+    "logmel_stream_windows": (_i, [_i64, _i, _i64, _i64, _vp, _i64, _i64p]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -155,6 +159,47 @@ def compute_noalloc(pcm, offsets, out, device_status=None, stream=None):
                                            _vp(out.data_ptr()), st, _stream_handle(stream, device)),
                "logmel_compute_noalloc")
     return out
+
+
+def encoder_chunks(frame_offsets, chunk_frames: int = 3000, quantum: int | None = None) -> np.ndarray:
+    """Offline encoder chunks over the rows of a log-mel batch
+    (logmel_encoder_chunks): int64 [n, 4] rows (utt, row, frames, padded).
+    frame_offsets are the batch's row offsets (Plan.frame_offsets).  Each
+    utterance's rows are cut into chunks of at most chunk_frames rows (3000 =
+    30 s), padded to a multiple of quantum rows (default chunk_frames: pad to
+    3000; smaller: length buckets).  Nothing is copied: see chunk_views."""
+    fo = _offsets(frame_offsets)
+    n_utt = fo.shape[0] - 1
+    q = chunk_frames if quantum is None else int(quantum)
+    count = int(_lib.logmel_encoder_chunk_count(_ptr64(fo), n_utt, int(chunk_frames)))
+    if count < 0:
+        _check(1, "logmel_encoder_chunk_count")
+    out = np.zeros((count, 4), dtype=np.int64)
+    n = ctypes.c_int64(0)
+    _check(_lib.logmel_encoder_chunks(_ptr64(fo), n_utt, int(chunk_frames), q, _vp(out.ctypes.data), count,
+                                      ctypes.byref(n)), "logmel_encoder_chunks")
+    return out
+
+
+def stream_windows(n_frames: int, finished: bool, chunk_frames: int = 500, context: int = 50) -> np.ndarray:
+    """Streaming encoder windows (logmel_stream_windows): int64 [n, 5] rows
+    (chunk, core_begin, core_end, ctx_begin, ctx_end) over a stream's frames,
+    for the chunks whose right context has arrived (all chunks once the
+    stream has finished)."""
+    n = ctypes.c_int64(0)
+    code = _lib.logmel_stream_windows(int(n_frames), int(bool(finished)), int(chunk_frames), int(context), None, 0,
+                                      ctypes.byref(n))
+    if code != 0 and n.value == 0:
+        _check(code, "logmel_stream_windows")
+    out = np.zeros((n.value, 5), dtype=np.int64)
+    _check(_lib.logmel_stream_windows(int(n_frames), int(bool(finished)), int(chunk_frames), int(context),
+                                      _vp(out.ctypes.data), n.value, ctypes.byref(n)), "logmel_stream_windows")
+    return out
+
+
+def chunk_views(out, chunks: np.ndarray) -> list:
+    """Zero-copy views out[row:row + frames] of the chunks' rows."""
+    return [out[int(r):int(r) + int(f)] for _, r, f, _ in chunks]
 
 
 class Plan:
