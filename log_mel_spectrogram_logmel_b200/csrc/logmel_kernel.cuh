@@ -5,15 +5,17 @@
 // samples -> symmetric Hamming window -> real DFT (201 bins) -> |X|^2 ->
 // 128 triangular mel filters -> ln(max(., 1e-10)).
 //
-// Structure (one persistent kernel, 160 threads, tiles of 32 frames; frame
-// slots d and d + 16 form the pair carried by one thread):
+// Structure (one persistent kernel; tile groups of 160 threads, up to three
+// per CTA, each working through tiles of 32 frames; frame slots d and d + 16
+// form the pair carried by one thread):
 //   stage   each tile's overlapping sample span is copied from HBM once into
-//           shared memory by the bulk-copy (TMA) engine: one 2-D tensor copy
-//           of 34 rows of 160 samples into 164-float slots when the span
-//           starts on a 160-sample row, else one bulk copy per hop block
-//           (cp.async when the source is not 16-byte aligned); a half-warp
-//           reads 8 frame pairs x 2 roles, so pass A's strided reads are
-//           conflict-free
+//           shared memory by the bulk-copy (TMA) engine, as 34 hop blocks of
+//           160 samples in 164-float slots, from the 16-byte boundary at or
+//           before the span (the slots then hold their samples from that
+//           shift): one 2-D tensor copy when the span starts on a 160-sample
+//           row, else one 3-D tensor copy over overlapping rows, else one
+//           bulk copy per hop block, else cp.async; a half-warp reads 8 frame
+//           pairs x 2 roles, so pass A's strided reads are conflict-free
 //   pass A  real FFT-400 as a complex FFT-200 of z[m] = x[2m] + i x[2m+1]
 //           (window applied on load), Cooley-Tukey 200 = 20 x 10: ten
 //           20-point DFTs per frame (prime-factor 4 x 5, no inner twiddles),
@@ -64,10 +66,9 @@ constexpr int MAX_WEIGHTS = 2 * NBINS;    // each bin feeds at most two triangle
 constexpr int CARRY_CAP = NFFT;           // carried samples per stream (< 400)
 constexpr int INLINE_UTT = 256;           // offline batches up to this size carry their metadata in the parameters
 
-// ln(1e-10) rounded to fp32: the value written wherever the mel energy is
-// below 1e-10 (section 2.3 step 5's floor).
+// ln(1e-10) rounded to fp32: the lower clamp of the logarithm (section 2.3
+// step 5's floor at mel energy 1e-10); zero energy gives exactly this value.
 constexpr float LOG_FLOOR = -23.025850929940457f;
-constexpr float ENERGY_FLOOR = 1e-10f;
 
 // FFT tables, built in float64 on the host by the plan and rounded to fp32;
 // one copy in shared memory serves every tile group of a CTA.
