@@ -80,3 +80,21 @@ def test_null_handles_are_rejected(cdll):
     cdll.logmel_plan_destroy(None)
     cdll.logmel_stream_destroy.argtypes = [ctypes.c_void_p]
     cdll.logmel_stream_destroy(None)
+
+
+def test_noalloc_limits_precede_cuda(cdll):
+    """The allocation-free entry point refuses batches beyond its fixed
+    scratch (4096 utterances, 32768 tiles) before any CUDA call."""
+    f = cdll.logmel_compute_noalloc
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int64), ctypes.c_int64] + [ctypes.c_void_p] * 3
+    import numpy as np
+    many = np.arange(4098, dtype=np.int64) * 400                     # 4097 utterances of one frame
+    assert f(ctypes.c_void_p(16), many.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), 4097, ctypes.c_void_p(16),
+             None, None) == 7
+    long_one = np.array([0, 32768 * 32 * 160 + 400], dtype=np.int64)  # 32769 tiles
+    assert f(ctypes.c_void_p(16), long_one.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), 1, ctypes.c_void_p(16),
+             None, None) == 7
+    bad = np.array([0, 10, 5], dtype=np.int64)                         # decreasing offsets
+    assert f(ctypes.c_void_p(16), bad.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), 2, ctypes.c_void_p(16),
+             None, None) == 1

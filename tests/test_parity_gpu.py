@@ -187,3 +187,21 @@ def test_errors_are_reported(lib, plan):
         lib.Plan(hop=100)
     assert e.value.code == 2
     assert plan.device_status() == 0
+
+
+def test_sizes_beyond_the_kernels_index_range_are_refused(lib, plan):
+    """Frame counts past int32 return LOGMEL_ERR_INPUT_TOO_LONG before any
+    work is enqueued (nothing is truncated); the buffers are never touched,
+    so small ones stand in for the huge input the offsets describe."""
+    import ctypes
+    x = torch.zeros(1024, device="cuda")
+    out = torch.zeros(16, 128, device="cuda")
+    for off in ([0, 160 * (2 ** 31) + 400], [0, 160 * (2 ** 30) + 400, 2 * 160 * (2 ** 30) + 800]):
+        o = np.ascontiguousarray(off, np.int64)
+        code = lib._lib.logmel_compute(plan._h, ctypes.c_void_p(x.data_ptr()),
+                                       o.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), len(off) - 1,
+                                       ctypes.c_void_p(out.data_ptr()), None)
+        assert code == 5, code
+    torch.cuda.synchronize()
+    assert not out.any()
+    assert plan.device_status() == 0
