@@ -11,6 +11,12 @@ library has not been built (``python log_mel_spectrogram_logmel_b200/build.py``)
 
     st = lm.Stream(plan, n_streams=1024)
     out, n = st.push_batch(chunks_cuda_f32)           # [1024, cap, 128], frames per stream
+
+    chunks = lm.encoder_chunks(plan.frame_offsets(offsets_int64))   # 3000-row encoder inputs
+    views = lm.chunk_views(out, chunks)                # zero-copy row views
+    windows = lm.stream_windows(frames_so_far, finished=False)      # 500-frame chunks, +-50 context
+
+    lm.compute_noalloc(pcm_cuda_f32, offsets_int64, out)  # no device allocation (fixed scratch)
 """
 from __future__ import annotations
 
