@@ -207,6 +207,75 @@ def run_reference(args, world, rank):
     return 0
 
 
+def compare_dft_gemm(args):
+    """The DFT as a dense GEMM (windowed frames [F, 400] x basis [400, 398],
+    the cos and sin rows of bins 1..199), timed with the library GEMM in fp32,
+    TF32 and 3xTF32 (three TF32 products of hi/lo splits, the split needed
+    for fp32-level accuracy), against the fused FFT kernel's whole step on
+    the same batch.  Measurement only: prints one JSON line."""
+    import torch
+    import log_mel_spectrogram_logmel_b200 as lm
+    dev = torch.device("cuda", 0)
+    pcm_h, off = rank_batch(0)
+    pcm = torch.from_numpy(pcm_h).to(dev)
+    frames = N_CLIPS * FRAMES_PER_CLIP
+    plan = lm.Plan(device=dev)
+    out = torch.empty((frames, N_MELS), dtype=torch.float32, device=dev)
+    n = torch.arange(400, dtype=torch.float64, device=dev)
+    win = (0.54 - 0.46 * torch.cos(2 * np.pi * n / 399)).float()
+    k = torch.arange(1, 200, dtype=torch.float64, device=dev)
+    ang = 2 * np.pi * torch.remainder(n[:, None] * k[None, :], 400) / 400
+    basis = torch.cat([torch.cos(ang), -torch.sin(ang)], 1).float().contiguous()   # [400, 398]
+    b_hi = basis.to(torch.bfloat16).float()                                          # coarse part
+    b_lo = basis - b_hi
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def frames_matrix():
+        views = [pcm[o:o + 160 * (FRAMES_PER_CLIP - 1) + 400].unfold(0, 400, 160) for o in off[:-1]]
+        return torch.cat(views) * win
+
+    def timed(fn, reps=20):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.fill_(1.0)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            ts.append((e0, e1))
+        torch.cuda.synchronize()
+        return sorted(a.elapsed_time(b) for a, b in ts)[reps // 2]
+
+    xw = frames_matrix()
+    x_hi = xw.to(torch.bfloat16).float()
+    x_lo = xw - x_hi
+    res = {"compare": "dft_gemm", "workload": WORKLOAD, "frames": frames,
+           "gemm_flop": 2 * frames * 400 * 398}
+    res["fused_kernel_step_ms"] = timed(lambda: plan.compute(pcm, off, out=out))
+    res["frames_materialise_ms"] = timed(frames_matrix)
+    torch.backends.cuda.matmul.allow_tf32 = False
+    res["gemm_fp32_ms"] = timed(lambda: xw @ basis)
+    torch.backends.cuda.matmul.allow_tf32 = True
+    res["gemm_tf32_ms"] = timed(lambda: xw @ basis)
+    res["gemm_3xtf32_ms"] = timed(lambda: x_hi @ b_hi + (x_hi @ b_lo + x_lo @ b_hi))
+    # accuracy of each product on a sample of frames, against the fp64 DFT:
+    # max |error| over the sample relative to each frame's largest coefficient
+    rows = torch.arange(0, frames, max(1, frames // 2048), device=dev)
+    want = xw[rows].double() @ (basis.double())
+    scale = want.abs().amax(1, keepdim=True).clamp_min(1e-30)
+    for name, f32 in (("fp32", False), ("tf32", True)):
+        torch.backends.cuda.matmul.allow_tf32 = f32
+        res["rel_err_" + name] = float(((xw[rows] @ basis).double() - want).abs().div(scale).max())
+    torch.backends.cuda.matmul.allow_tf32 = True
+    got = x_hi[rows] @ b_hi + (x_hi[rows] @ b_lo + x_lo[rows] @ b_hi)
+    res["rel_err_3xtf32"] = float((got.double() - want).abs().div(scale).max())
+    torch.backends.cuda.matmul.allow_tf32 = False
+    print(json.dumps(res), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -215,7 +284,11 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    ap.add_argument("--compare", choices=["dft-gemm"], default=None,
+                    help="time the DFT as a library GEMM against the fused kernel (one GPU, no bench line)")
     args = ap.parse_args()
+    if args.compare == "dft-gemm":
+        return compare_dft_gemm(args)
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_env()
     if args.impl == "reference":
