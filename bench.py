@@ -276,6 +276,66 @@ def compare_dft_gemm(args):
     return 0
 
 
+def compare_workloads(args):
+    """The other workloads, timed one call at a time (median of CUDA-event
+    timings, L2 flushed before each): the ragged batch of 256 utterances of
+    U[1 s, 30 s], the 87-minute long-form recording as 174 chunks of 30 s
+    plus its tail, the dense bench batch, and a streaming push of 80 ms to
+    each of 1024 streams.  Measurement only: prints one JSON line per workload."""
+    import torch
+    import log_mel_spectrogram_logmel_b200 as lm
+    dev = torch.device("cuda", 0)
+    plan = lm.Plan(device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def median_ms(fn, reps):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.fill_(1.0)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            ts.append((e0, e1))
+        torch.cuda.synchronize()
+        return sorted(a.elapsed_time(b) for a, b in ts)[reps // 2]
+
+    def offline(name, pcm_h, off, reps):
+        x = torch.from_numpy(pcm_h).to(dev)
+        frames = int(plan.frame_offsets(off)[-1])
+        out = torch.empty((frames, N_MELS), dtype=torch.float32, device=dev)
+        ms = median_ms(lambda: plan.compute(x, off, out=out), reps)
+        print(json.dumps({"compare": "workloads", "workload": name, "n_utt": len(off) - 1, "frames": frames,
+                          "ms_per_call": ms, "frames_per_s": frames / (ms / 1e3)}), flush=True)
+
+    offline("dense batch: 64 clips x 30 s", *rank_batch(0), reps=50)
+    offline("ragged batch: 256 utterances, lengths U[1 s, 30 s]", *W.ragged_batch(), reps=50)
+    offline("long-form: 87 min recording (20% silent segments) as 30 s chunks", *W.long_form(), reps=20)
+
+    n_streams, push = 1024, 1280                        # 80 ms at 16 kHz
+    sig = torch.from_numpy(W.stream_signals(n_streams, n_samples=push * 8)).to(dev)
+    st = lm.Stream(plan, n_streams)
+    # a push emits at most this many frames once the carries hold up to 399 samples
+    out = torch.empty((n_streams, (push + 399) // 160 + 1, N_MELS), dtype=torch.float32, device=dev)
+    for j in range(4):                                  # fill the carries: steady state
+        st.push_batch(sig[:, j * push:(j + 1) * push], out=out)
+    k, emitted = [4], [0]
+
+    def one_push():
+        j = k[0] % 8
+        _, n = st.push_batch(sig[:, j * push:(j + 1) * push], out=out)
+        emitted[0] = int(n.sum())
+        k[0] += 1
+    ms = median_ms(one_push, 200)
+    frames = emitted[0]
+    print(json.dumps({"compare": "workloads", "workload": "streaming push: 1024 streams x 80 ms",
+                      "frames": frames, "ms_per_call": ms, "frames_per_s": frames / (ms / 1e3),
+                      "audio_s_per_s": n_streams * push / W.SR / (ms / 1e3)}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -284,11 +344,14 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
-    ap.add_argument("--compare", choices=["dft-gemm"], default=None,
-                    help="time the DFT as a library GEMM against the fused kernel (one GPU, no bench line)")
+    ap.add_argument("--compare", choices=["dft-gemm", "workloads"], default=None,
+                    help="dft-gemm: the DFT as a library GEMM against the fused kernel; "
+                         "workloads: the ragged, long-form and streaming workloads (one GPU, no bench line)")
     args = ap.parse_args()
     if args.compare == "dft-gemm":
         return compare_dft_gemm(args)
+    if args.compare == "workloads":
+        return compare_workloads(args)
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_env()
     if args.impl == "reference":
