@@ -290,9 +290,14 @@ class Stream:
             self._h = None
 
     def frames_for_push(self, stream_id: int, length: int) -> int:
+        """Frames the next push of `length` samples to one stream emits."""
         return int(_lib.logmel_stream_frames_for_push(self._h, stream_id, int(length)))
 
     def max_frames(self, length: int) -> int:
+        """Largest per-stream count the NEXT push_batch of `length` samples
+        emits; it grows as the carries fill (a carry holds at most n_fft - 1
+        samples), so a buffer reused across pushes is sized with
+        (length - 1) // hop + 1 rows, the count for a full carry."""
         return int(_lib.logmel_stream_max_frames(self._h, int(length)))
 
     def push(self, stream_id: int, chunk, out=None, stream=None):

@@ -99,7 +99,11 @@ def test_streams_in_different_states(plan, lib):
     for _ in range(20):
         for s in range(S):
             chunk[s] = x[s, pos[s]:pos[s] + L]
+        expect = [st.frames_for_push(s, L) for s in range(S)]
+        # the next push's largest count; a full carry (n_fft - 1 samples) bounds it
+        assert st.max_frames(L) == max(expect) <= (L - 1) // 160 + 1
         o, n = st.push_batch(chunk)
+        assert n.tolist() == expect
         for s in range(S):
             outs[s].append(o[s, :n[s]].clone())
         pos += L
