@@ -310,9 +310,15 @@ def compare_workloads(args):
         print(json.dumps({"compare": "workloads", "workload": name, "n_utt": len(off) - 1, "frames": frames,
                           "ms_per_call": ms, "frames_per_s": frames / (ms / 1e3)}), flush=True)
 
-    offline("dense batch: 64 clips x 30 s", *rank_batch(0), reps=50)
-    offline("ragged batch: 256 utterances, lengths U[1 s, 30 s]", *W.ragged_batch(), reps=50)
-    offline("long-form: 87 min recording (20% silent segments) as 30 s chunks", *W.long_form(), reps=20)
+    only = args.only
+    if only in (None, "dense"):
+        offline("dense batch: 64 clips x 30 s", *rank_batch(0), reps=50)
+    if only in (None, "ragged"):
+        offline("ragged batch: 256 utterances, lengths U[1 s, 30 s]", *W.ragged_batch(), reps=50)
+    if only in (None, "long-form"):
+        offline("long-form: 87 min recording (20% silent segments) as 30 s chunks", *W.long_form(), reps=20)
+    if only not in (None, "streaming"):
+        return 0
 
     n_streams, push = 1024, 1280                        # 80 ms at 16 kHz
     sig = torch.from_numpy(W.stream_signals(n_streams, n_samples=push * 8)).to(dev)
@@ -347,6 +353,8 @@ def main():
     ap.add_argument("--compare", choices=["dft-gemm", "workloads"], default=None,
                     help="dft-gemm: the DFT as a library GEMM against the fused kernel; "
                          "workloads: the ragged, long-form and streaming workloads (one GPU, no bench line)")
+    ap.add_argument("--only", choices=["dense", "ragged", "long-form", "streaming"], default=None,
+                    help="with --compare workloads: time this workload alone")
     args = ap.parse_args()
     if args.compare == "dft-gemm":
         return compare_dft_gemm(args)

@@ -660,8 +660,10 @@ __device__ __forceinline__ void stage_tile(Ctl& S, float* span, int tid, const A
       for (int q = 0; q < (31 * HOP + NFFT + HOP - 1) / HOP; ++q)
         if (tid + HOP * q < n) cp_async4(dst + BLK * q + tid, base + tid + HOP * q);
     } else {
+      // streaming (carry ++ chunk): a push stages far fewer samples than the
+      // span holds, so the loop runs over the staged hop blocks only
 #pragma unroll 2
-      for (int q = 0; q < (31 * HOP + NFFT + HOP - 1) / HOP; ++q) {
+      for (int q = 0; HOP * q < n; ++q) {
         const int64_t pos = g.start + tid + HOP * q;
         if (tid + HOP * q < n)
           cp_async4(dst + BLK * q + tid, pos < g.len0 ? g.src0 + pos : g.src1 + (pos - g.len0));
