@@ -184,3 +184,31 @@ def test_streaming_full_size_1024x600(plan, lib):
         L_, M_ = O.log_mel_frames(xh[s], [0, N], rows)
         check_against_oracle(got[s].cpu().numpy()[rows], L_, M_)
     assert plan.device_status() == 0
+
+
+def test_long_form_streamed_equals_offline_whole_recording(plan, lib):
+    # the 87-minute recording pushed through one stream in pieces from one
+    # sample to 3 M samples equals the offline log-mel of the whole recording
+    # taken as one utterance: 521,998 frames (continuous, not cut at 30 s)
+    pcm, _ = W.long_form()
+    N = pcm.shape[0]
+    x = torch.from_numpy(pcm).cuda()
+    rng = np.random.default_rng(44)
+    st = lib.Stream(plan, 1)
+    outs, pos = [], 0
+    while pos < N:
+        L = int(rng.integers(1, 3_000_000)) if rng.random() < 0.7 else int(rng.integers(1, 2000))
+        L = min(L, N - pos)
+        n_expect = st.frames_for_push(0, L)
+        o = st.push(0, x[pos:pos + L])
+        assert o.shape[0] == n_expect
+        outs.append(o)
+        pos += L
+    got = torch.cat(outs, 0)
+    assert got.shape == (O.num_frames(N), 128) == (521_998, 128)
+    ref = plan.compute(x, [0, N])
+    assert torch.equal(_bits(got), _bits(ref))
+    rows = np.sort(rng.choice(got.shape[0], 400, replace=False))
+    L_, M_ = O.log_mel_frames(pcm, [0, N], rows)
+    check_against_oracle(got.cpu().numpy()[rows], L_, M_)
+    assert plan.device_status() == 0
