@@ -142,7 +142,11 @@ logmel_status logmel_stream_push_batch(logmel_stream* st, const float* chunks, i
                                        int64_t len, float* out, int64_t out_capacity,
                                        int64_t* n_frames_out, void* stream);
 
-/* Largest per-stream frame count the next push_batch of `len` samples emits. */
+/* Largest per-stream frame count the next push_batch of `len` samples emits.
+ * It depends on the carries' current lengths (it grows as they fill); a
+ * carry never holds more than n_fft - 1 samples, so (len - 1) / hop + 1
+ * (integer division, len >= 1) bounds the count in every state, which is
+ * the size for an output buffer reused across pushes. */
 int64_t logmel_stream_max_frames(const logmel_stream* st, int64_t len);
 
 /* Checkpoint / resume of the carry state.  logmel_stream_state_bytes gives
