@@ -203,10 +203,21 @@ logmel_status logmel_stream_reset(logmel_stream* st, int stream_id, void* stream
  * them on one stream or with events.  Host-side, calls are serialised by a
  * lock.  Each call clears the status word and launches one kernel; batches
  * of more than 256 utterances first copy their metadata host->device from a
- * static host buffer with cudaMemcpyAsync.  No device or pinned memory is
- * allocated or freed. */
+ * static host buffer with cudaMemcpyAsync.  That buffer is pageable host
+ * memory, so such a call may block the calling thread until `stream` has
+ * reached the copy (a copy from pageable memory returns once its source has
+ * been consumed), and the next call rewrites the buffer.  Batches of up to
+ * 256 utterances carry their metadata in the kernel launch and do not block.
+ * No device or pinned memory is allocated or freed. */
 logmel_status logmel_compute_noalloc(const float* pcm, const int64_t* offsets, int64_t n_utt,
                                      float* out, int* device_status, void* stream);
+
+/* Output rows logmel_compute_noalloc writes for these offsets: the sum over
+ * utterances of floor((len_u - 400) / 160) + 1 (0 for len_u < 400), the frame
+ * count of section 2.3 step 1 for the default front-end.  Host only, needs
+ * no plan and no device; -1 for NULL offsets, n_utt < 0 or decreasing
+ * offsets. */
+int64_t logmel_noalloc_total_frames(const int64_t* offsets, int64_t n_utt);
 
 /* ---- Encoder-ready index maps over the log-mel rows (host only) ----------
  * The steps right after the log-mel front-end cut its rows into encoder
@@ -267,6 +278,32 @@ typedef struct {
  * LOGMEL_ERR_INVALID_ARG is returned. */
 logmel_status logmel_stream_windows(int64_t n_frames, int finished, int64_t chunk_frames, int64_t context,
                                     logmel_window* windows, int64_t capacity, int64_t* n_windows);
+
+/* ---- Data-parallel split over ranks (host only) ----------------------------
+ * Every frame reads only its own 400 samples (section 2.3 step 1), so the
+ * utterances of one batch, or a set of streams, are split over GPUs with no
+ * data exchanged between them: each rank runs logmel_compute (or its pushes)
+ * on its own part, on its own device.
+ *
+ * logmel_partition_utterances: frame_offsets (host, n_utt + 1 entries, as
+ * logmel_frame_offsets returns them, non-decreasing) -> utt_begin (host,
+ * n_parts + 1 entries).  Rank r takes the contiguous utterances
+ * utt_begin[r] .. utt_begin[r + 1] - 1, i.e. samples offsets[utt_begin[r]] ..
+ * offsets[utt_begin[r + 1]] and output rows frame_offsets[utt_begin[r]] ..
+ * frame_offsets[utt_begin[r + 1]] of the whole batch.  The cut before rank r
+ * is the utterance boundary whose frame prefix sum is nearest to r / n_parts
+ * of the batch's frames (the smaller index on a tie), so each rank's frame
+ * count is within one utterance's frames of the mean.  Ranks may be empty.
+ * LOGMEL_ERR_INVALID_ARG on NULL pointers, n_utt < 0, n_parts < 1 or
+ * decreasing offsets; LOGMEL_ERR_INPUT_TOO_LONG if n_parts times the frame
+ * count overflows.
+ *
+ * logmel_partition_streams: stream ids 0 .. n_streams - 1 -> stream_begin
+ * (host, n_parts + 1 entries): rank r takes ids floor(r S / G) ..
+ * floor((r + 1) S / G) - 1, runs whose sizes differ by at most one. */
+logmel_status logmel_partition_utterances(const int64_t* frame_offsets, int64_t n_utt, int n_parts,
+                                          int64_t* utt_begin);
+logmel_status logmel_partition_streams(int64_t n_streams, int n_parts, int64_t* stream_begin);
 
 /* Reads and clears the plan's device status word (synchronises `stream`).
  * *code = 0 when no kernel has flagged an inconsistency since the last read. */

@@ -26,7 +26,7 @@ import os
 import numpy as np
 
 __all__ = ["Plan", "Stream", "LogMelError", "compute_noalloc", "encoder_chunks", "stream_windows", "chunk_views",
-           "lib_path", "exported_symbols", "STATUS"]
+           "partition_utterances", "partition_streams", "lib_path", "exported_symbols", "STATUS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "liblogmel_b200.so")
@@ -67,6 +67,7 @@ _SIGS = {
     "logmel_total_frames": (_i64, [_p, _i64p, _i64]),
     "logmel_compute": (_i, [_p, _vp, _i64p, _i64, _vp, _vp]),
     "logmel_compute_noalloc": (_i, [_vp, _i64p, _i64, _vp, _vp, _vp]),
+    "logmel_noalloc_total_frames": (_i64, [_i64p, _i64]),
     "logmel_stream_create": (_i, [_p, _i, ctypes.POINTER(_p)]),
     "logmel_stream_destroy": (None, [_p]),
     "logmel_stream_frames_for_push": (_i64, [_p, _i, _i64]),
@@ -81,6 +82,8 @@ _SIGS = {
     "logmel_encoder_chunk_count": (_i64, [_i64p, _i64, _i64]),
     "logmel_encoder_chunks": (_i, [_i64p, _i64, _i64, _i64, _vp, _i64, _i64p]),
     "logmel_stream_windows": (_i, [_i64, _i, _i64, _i64, _vp, _i64, _i64p]),
+    "logmel_partition_utterances": (_i, [_i64p, _i64, _i, _i64p]),
+    "logmel_partition_streams": (_i, [_i64, _i, _i64p]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -148,10 +151,9 @@ def compute_noalloc(pcm, offsets, out, device_status=None, stream=None):
     off = _offsets(offsets)
     if off[-1] > pcm.numel():
         raise ValueError("offsets reach beyond pcm")
-    n = np.diff(off)
-    if np.any(n < 0) or off[0] < 0:
+    total = int(_lib.logmel_noalloc_total_frames(_ptr64(off), off.shape[0] - 1))
+    if total < 0:
         raise ValueError("offsets must be non-negative and non-decreasing")
-    total = int(np.where(n >= 400, (n - 400) // 160 + 1, 0).sum())
     if out.numel() < total * 128:
         raise ValueError("out is too small")
     st = _vp(0)
@@ -200,6 +202,26 @@ def stream_windows(n_frames: int, finished: bool, chunk_frames: int = 500, conte
     out = np.zeros((n.value, 5), dtype=np.int64)
     _check(_lib.logmel_stream_windows(int(n_frames), int(bool(finished)), int(chunk_frames), int(context),
                                       _vp(out.ctypes.data), n.value, ctypes.byref(n)), "logmel_stream_windows")
+    return out
+
+
+def partition_utterances(frame_offsets, n_parts: int) -> np.ndarray:
+    """Data-parallel split of a batch (logmel_partition_utterances): int64
+    utt_begin [n_parts + 1]; rank r takes utterances utt_begin[r] ..
+    utt_begin[r + 1] - 1 and writes rows frame_offsets[utt_begin[r]] ..
+    frame_offsets[utt_begin[r + 1]] of the batch, balanced by frame count."""
+    fo = _offsets(frame_offsets)
+    out = np.zeros(int(n_parts) + 1, dtype=np.int64)
+    _check(_lib.logmel_partition_utterances(_ptr64(fo), fo.shape[0] - 1, int(n_parts), _ptr64(out)),
+           "logmel_partition_utterances")
+    return out
+
+
+def partition_streams(n_streams: int, n_parts: int) -> np.ndarray:
+    """Stream ids split over ranks (logmel_partition_streams): int64
+    stream_begin [n_parts + 1]; rank r takes ids stream_begin[r] .. stream_begin[r + 1] - 1."""
+    out = np.zeros(int(n_parts) + 1, dtype=np.int64)
+    _check(_lib.logmel_partition_streams(int(n_streams), int(n_parts), _ptr64(out)), "logmel_partition_streams")
     return out
 
 

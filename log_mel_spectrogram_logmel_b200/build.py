@@ -14,7 +14,8 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "liblogmel_b200.so")
-SOURCES = [os.path.join(PKG, "csrc", "logmel.cu"), os.path.join(PKG, "csrc", "chunk_map.cpp")]
+SOURCES = [os.path.join(PKG, "csrc", "logmel.cu"), os.path.join(PKG, "csrc", "chunk_map.cpp"),
+           os.path.join(PKG, "csrc", "partition.cpp")]
 DEPS = SOURCES + [os.path.join(PKG, "csrc", "logmel_kernel.cuh"), os.path.join(PKG, "csrc", "mel_layout_default.h"),
                   os.path.join(ROOT, "include", "logmel.h")]
 

@@ -965,6 +965,13 @@ static logmel_status noalloc_setup(int dev, NoAllocDevice& d) {
   return LOGMEL_OK;
 }
 
+extern "C" int64_t logmel_noalloc_total_frames(const int64_t* off, int64_t n_utt) {
+  if (check_offsets(off, n_utt) != LOGMEL_OK) return -1;
+  int64_t t = 0;
+  for (int64_t u = 0; u < n_utt; ++u) t += frames_of(off[u + 1] - off[u]);
+  return t;
+}
+
 extern "C" logmel_status logmel_compute_noalloc(const float* pcm, const int64_t* off, int64_t n_utt,
                                                  float* out, int* device_status, void* stream) {
   logmel_status st = check_offsets(off, n_utt);

@@ -98,3 +98,24 @@ def test_noalloc_limits_precede_cuda(cdll):
     bad = np.array([0, 10, 5], dtype=np.int64)                         # decreasing offsets
     assert f(ctypes.c_void_p(16), bad.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), 2, ctypes.c_void_p(16),
              None, None) == 1
+
+
+def test_noalloc_total_frames_is_the_frame_count(cdll):
+    """The plan-free row count of the allocation-free entry point equals the
+    oracle's frame count (section 2.3 step 1) on ragged lengths around the
+    400-sample frame and the 160-sample hop, and refuses bad offsets."""
+    import numpy as np
+
+    import oracle as O
+    f = cdll.logmel_noalloc_total_frames
+    f.restype = ctypes.c_int64
+    f.argtypes = [ctypes.POINTER(ctypes.c_int64), ctypes.c_int64]
+    lens = [0, 1, 399, 400, 401, 559, 560, 561, 16000, 480000, 83_520_000]
+    off = 7 + np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    p64 = off.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))
+    assert f(p64, len(lens)) == O.frame_offsets(off)[-1] == sum(O.num_frames(n) for n in lens)
+    assert f(p64, 0) == 0
+    bad = np.array([0, 10, 5], dtype=np.int64)
+    assert f(bad.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), 2) == -1
+    assert f(None, 1) == -1
+    assert f(p64, -1) == -1

@@ -30,7 +30,7 @@ def _rank_main(rank, world, port, q):
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
-        pcm, off = bench.rank_batch(rank, n_clips=2)
+        pcm, off = bench.rank_batch(rank, world, n_clips=2)
         local_ms = 10.0 + 5.0 * rank                     # rank 1 is the slow one
         total_ms = bench.reduce_max(dist, local_ms, torch.device("cpu"))
         frames = 2 * bench.FRAMES_PER_CLIP
