@@ -63,17 +63,38 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def ncu_traffic():
-    """DRAM bytes per launch of the fused kernel from the committed ncu summary,
-    if it was taken on the current kernel source; else None."""
+FLOP_PER_FRAME = 400 + 8644 + 603 + 790 + 128   # window, rFFT-400 (2.5 N log2 N), power, mel, log
+
+
+def ncu_counters():
+    """The fused kernel's counters from the committed ncu summary, if they were
+    taken on the current kernel source; else an empty dict."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(path):
-        return None
+        return {}
     with open(path) as f:
         d = json.load(f)
     if d.get("kernel_source_hash") != kernel_source_hash():
-        return None
-    return d.get("dram_bytes_per_launch_full_step")
+        return {}
+    return d
+
+
+def fp32_peak_tflops():
+    """The FP32 roof measured on this device: the FMA probe library's better
+    rate of the packed (f32x2) and scalar forms, 2 flops per FMA lane-op."""
+    import ctypes
+    path = os.path.join(ROOT, "log_mel_spectrogram_logmel_b200", "libfp32_peak.so")
+    lib = ctypes.CDLL(path)
+    lib.fp32_fma_probe.restype = ctypes.c_int
+    lib.fp32_fma_probe.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_double)]
+    best = {}
+    for packed in (1, 0):
+        r = ctypes.c_double(0.0)
+        rc = lib.fp32_fma_probe(packed, 4, 20000, ctypes.byref(r))
+        if rc != 0:
+            raise RuntimeError(f"fp32_fma_probe failed: cudaError {rc}")
+        best["packed" if packed else "scalar"] = 2 * r.value / 1e12
+    return max(best.values()), best
 
 
 class ClockSampler:
@@ -471,6 +492,9 @@ def main():
         achieved = bytes_launch / (ms_per_step / 1e3) / 1e9
         peak = float(peaks["hbm_gbs"])
         cpu_value, cores, sample = cpu_oracle_rate(args.cpu_budget_s, FRAMES_PER_CLIP) if world == 1 else (None, None, None)
+        nc = ncu_counters()
+        fp32_peak, fp32_forms = fp32_peak_tflops()
+        fp32_achieved = FLOP_PER_FRAME * frames / (ms_per_step / 1e3) / 1e12
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -482,11 +506,23 @@ def main():
                        "parallelism": f"dp{world} (the job's world x 64 clips split by the frame-balanced "
                                       f"partition of utterances; no collective on the data path)"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": ncu_traffic(),
+                         "frac": achieved / peak, "traffic": nc.get("dram_bytes_per_launch_full_step"),
+                         "traffic_read": nc.get("dram_bytes_read"), "traffic_write": nc.get("dram_bytes_write"),
+                         "traffic_note": "DRAM bytes counted during one launch (ncu, same kernel source); part "
+                                         "of the rows written is still in L2 when the kernel ends and reaches "
+                                         "DRAM later, so the write count is below the rows' bytes",
                          "peak_source": f"{peak_kind} hbm_gbs (burst copy)",
                          "algorithmic_bytes_per_launch": bytes_launch,
                          "kernel": "logmel_fused_kernel (1 launch per step; the event pair brackets the "
-                                   "call, whose batch index map travels in the launch parameters)"},
+                                   "call, whose batch index map travels in the launch parameters)",
+                         "fp32": {"achieved": fp32_achieved, "peak": fp32_peak, "unit": "TFLOP/s",
+                                  "frac": fp32_achieved / fp32_peak, "flop_per_frame": FLOP_PER_FRAME,
+                                  "peak_source": "measured this run: FMA probe (libfp32_peak), best of "
+                                                 + ", ".join(f"{k} {v:.1f}" for k, v in fp32_forms.items()),
+                                  "fma_pipe_active_pct": nc.get("fma_pipe_active_pct"),
+                                  "issue_active_pct": nc.get("issue_active_pct"),
+                                  "shared_wavefronts_per_frame": nc.get("shared_wavefronts_per_frame"),
+                                  "inst_per_frame": nc.get("inst_per_frame")}},
             "cpu_baseline": ({"value": cpu_value, "unit": UNIT, "cores": cores, "kind": "oracle",
                               "sample": sample} if cpu_value else None),
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": 4 * n_samples,

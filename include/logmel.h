@@ -114,7 +114,9 @@ logmel_status logmel_compute(logmel_plan* plan, const float* pcm, const int64_t*
 int64_t logmel_total_frames(const logmel_plan* plan, const int64_t* offsets, int64_t n_utt);
 
 /* Streaming state for n_streams independent streams (device carry of up to
- * n_fft - 1 samples per stream; zero-initialised: every stream is empty). */
+ * n_fft - 1 samples per stream; zero-initialised: every stream is empty).
+ * The call synchronises the device once, so that the zeroed state is in
+ * place before it returns. */
 logmel_status logmel_stream_create(logmel_plan* plan, int n_streams, logmel_stream** out);
 void logmel_stream_destroy(logmel_stream* st);
 
@@ -141,6 +143,34 @@ logmel_status logmel_stream_push(logmel_stream* st, int stream_id, const float* 
 logmel_status logmel_stream_push_batch(logmel_stream* st, const float* chunks, int64_t chunk_stride,
                                        int64_t len, float* out, int64_t out_capacity,
                                        int64_t* n_frames_out, void* stream);
+
+/* Pushes a chunk of its own length to every stream at once, in one launch
+ * (chunked streaming input arriving as it comes: section 6 of the first
+ * page; the 80 / 120 / 160 ms audio clocks of the "Audio8-ASR-Infinite" page
+ * with streams whose pieces differ in size).
+ *   chunks         device, fp32, the pushed samples of all streams packed:
+ *                  stream s's chunk is chunks[chunk_offsets[s] ..
+ *                  chunk_offsets[s + 1]) (may be empty: the stream is left
+ *                  as it is)
+ *   chunk_offsets  host, int64 [n_streams + 1], non-decreasing, >= 0
+ *   out            device, fp32 [n_streams, out_capacity, n_mels]; stream s
+ *                  writes its n_frames_out[s] rows at out + s*out_capacity*n_mels
+ *   n_frames_out   host, int64 [n_streams], filled before the call returns
+ * Every stream s advances by its own chunk_offsets[s + 1] - chunk_offsets[s]
+ * samples; its output equals the offline log-mel of its concatenated audio
+ * bit for bit, as for the other pushes.  The offsets are copied
+ * host->device on `stream` through a pinned ring owned by the stream object
+ * (allocated on the first ragged push; the host thread waits only when it
+ * reuses a ring slot whose copy, four pushes earlier, is still pending).
+ * Returns LOGMEL_ERR_INVALID_ARG if any stream would emit more than
+ * out_capacity frames or the offsets are bad (nothing enqueued). */
+logmel_status logmel_stream_push_batch_ragged(logmel_stream* st, const float* chunks,
+                                              const int64_t* chunk_offsets, float* out,
+                                              int64_t out_capacity, int64_t* n_frames_out, void* stream);
+
+/* Largest per-stream frame count the next push_batch_ragged with these
+ * chunk_offsets (host, int64 [n_streams + 1]) emits; -1 on a bad argument. */
+int64_t logmel_stream_max_frames_ragged(const logmel_stream* st, const int64_t* chunk_offsets);
 
 /* Largest per-stream frame count the next push_batch of `len` samples emits.
  * It depends on the carries' current lengths (it grows as they fill); a
@@ -304,6 +334,20 @@ logmel_status logmel_stream_windows(int64_t n_frames, int finished, int64_t chun
 logmel_status logmel_partition_utterances(const int64_t* frame_offsets, int64_t n_utt, int n_parts,
                                           int64_t* utt_begin);
 logmel_status logmel_partition_streams(int64_t n_streams, int n_parts, int64_t* stream_begin);
+
+/* Test hook for the bounded wait on a tile's span copies (not for normal
+ * use; no page defines it).  Offline tiles staged by bulk copies wait on a
+ * shared-memory barrier, polling at most poll_limit times (0: the default
+ * 65536 polls, about 65 ms); a wait that runs out stores
+ * LOGMEL_DEVICE_COPY_TIMEOUT (3) in the plan's device status word, waits once
+ * more (again bounded) for the copies still in flight, and ends that tile
+ * group's work, so the call returns and the context stays usable (the
+ * group's remaining rows are not written).  extra_tx_bytes (a multiple of 16,
+ * at most 1 MiB) is added to the bytes each tile's barrier expects: every
+ * real copy is still issued and lands, but the barrier never completes, so
+ * the wait runs out.  (0, 0) restores normal operation.  Host only. */
+#define LOGMEL_DEVICE_COPY_TIMEOUT 3
+logmel_status logmel_plan_set_wait_test(logmel_plan* plan, int extra_tx_bytes, int poll_limit);
 
 /* Reads and clears the plan's device status word (synchronises `stream`).
  * *code = 0 when no kernel has flagged an inconsistency since the last read. */

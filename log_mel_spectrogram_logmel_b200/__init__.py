@@ -74,11 +74,14 @@ _SIGS = {
     "logmel_stream_push": (_i, [_p, _i, _vp, _i64, _vp, _i64, _i64p, _vp]),
     "logmel_stream_push_batch": (_i, [_p, _vp, _i64, _i64, _vp, _i64, _i64p, _vp]),
     "logmel_stream_max_frames": (_i64, [_p, _i64]),
+    "logmel_stream_push_batch_ragged": (_i, [_p, _vp, _i64p, _vp, _i64, _i64p, _vp]),
+    "logmel_stream_max_frames_ragged": (_i64, [_p, _i64p]),
     "logmel_stream_state_bytes": (_i64, [_p]),
     "logmel_stream_get_state": (_i, [_p, _vp, _i64, _vp]),
     "logmel_stream_set_state": (_i, [_p, _vp, _i64, _vp]),
     "logmel_stream_reset": (_i, [_p, _i, _vp]),
     "logmel_plan_device_status": (_i, [_p, ctypes.POINTER(_i), _vp]),
+    "logmel_plan_set_wait_test": (_i, [_p, _i, _i]),
     "logmel_encoder_chunk_count": (_i64, [_i64p, _i64, _i64]),
     "logmel_encoder_chunks": (_i, [_i64p, _i64, _i64, _i64, _vp, _i64, _i64p]),
     "logmel_stream_windows": (_i, [_i64, _i, _i64, _i64, _vp, _i64, _i64p]),
@@ -285,6 +288,13 @@ class Plan:
                "logmel_compute")
         return out
 
+    def set_wait_test(self, extra_tx_bytes: int, poll_limit: int) -> None:
+        """Test hook (logmel_plan_set_wait_test): make the bounded wait on
+        each tile's span copies run out (extra expected bytes that never
+        arrive, at most poll_limit polls); (0, 0) restores normal operation."""
+        _check(_lib.logmel_plan_set_wait_test(self._h, int(extra_tx_bytes), int(poll_limit)),
+               "logmel_plan_set_wait_test")
+
     def device_status(self, stream=None) -> int:
         code = ctypes.c_int(0)
         _check(_lib.logmel_plan_device_status(self._h, ctypes.byref(code), _stream_handle(stream, self.device)),
@@ -364,6 +374,37 @@ class Stream:
                                              _vp(out.data_ptr()), cap, _ptr64(n),
                                              _stream_handle(stream, self.plan.device)),
                "logmel_stream_push_batch")
+        return out, n
+
+    def push_batch_ragged(self, chunks, offsets, out=None, stream=None):
+        """Push chunks[offsets[s]:offsets[s + 1]] to every stream s, each its
+        own length (0 leaves a stream as it is), in one launch.  chunks is a
+        1-D CUDA float32 tensor, offsets host int64 [n_streams + 1].  Returns
+        (out [n_streams, cap, n_mels], n_frames int64 numpy [n_streams])."""
+        torch = _torch()
+        _check_cuda_f32(chunks, "chunks", self.plan.device)
+        off = _offsets(offsets)
+        if off.shape[0] != self.n_streams + 1:
+            raise ValueError("offsets must hold n_streams + 1 entries")
+        if off[-1] > chunks.numel():
+            raise ValueError("offsets reach beyond chunks")
+        need = int(_lib.logmel_stream_max_frames_ragged(self._h, _ptr64(off)))
+        if need < 0:
+            raise ValueError("offsets must be non-negative and non-decreasing")
+        nm = self.plan.n_mels
+        if out is None:
+            out = torch.empty((self.n_streams, max(need, 1), nm), dtype=torch.float32, device=self.plan.device)
+        if (not isinstance(out, torch.Tensor) or not out.is_cuda or out.dtype != torch.float32
+                or out.dim() != 3 or out.shape[0] != self.n_streams or out.shape[2] != nm
+                or out.stride(2) != 1 or out.stride(1) != nm or out.stride(0) % nm):
+            raise ValueError("out must be a [n_streams, frames, n_mels] float32 CUDA view with n_mels-contiguous rows")
+        if out.shape[1] < need:
+            raise ValueError(f"out holds {out.shape[1]} frames per stream, the push emits up to {need}")
+        n = np.zeros(self.n_streams, np.int64)
+        _check(_lib.logmel_stream_push_batch_ragged(self._h, _vp(chunks.data_ptr()), _ptr64(off),
+                                                    _vp(out.data_ptr()), out.stride(0) // nm, _ptr64(n),
+                                                    _stream_handle(stream, self.plan.device)),
+               "logmel_stream_push_batch_ragged")
         return out, n
 
     def state_bytes(self) -> int:

@@ -41,6 +41,24 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(p) <= t for p in DEPS)
 
 
+PEAK_LIB = os.path.join(PKG, "libfp32_peak.so")
+PEAK_SRC = os.path.join(PKG, "csrc", "fp32_peak.cu")
+
+
+def build_peak_probe(force: bool = False) -> str:
+    """The FP32 FMA probe that bench.py measures the FP32 roof with."""
+    if not force and os.path.exists(PEAK_LIB) and os.path.getmtime(PEAK_LIB) >= max(
+            os.path.getmtime(PEAK_SRC), os.path.getmtime(os.path.join(ROOT, "include", "fp32_peak.h"))):
+        return PEAK_LIB
+    cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-Xcompiler", "-fPIC",
+           "-shared", "-I", os.path.join(ROOT, "include"), "-o", PEAK_LIB + ".tmp", PEAK_SRC]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
+    os.replace(PEAK_LIB + ".tmp", PEAK_LIB)
+    return PEAK_LIB
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB
@@ -58,3 +76,4 @@ def build(force: bool = False, verbose: bool = False) -> str:
 
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose=True))
+    print(build_peak_probe(force="--force" in sys.argv))

@@ -93,40 +93,50 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// The PCM as a 3-D tensor [rows][40][w] whose element (x, y, z) is
-// pcm[160 z + 4 y + x]: rows of w samples start at every 16-byte boundary
-// (for w = 164 the strides overlap on purpose), so one 164 x 1 x 34 box
-// lands any tile's span, from the boundary at or before it, in its
-// hop-block slots.  Rows are counted so that every row of every start class
-// lies inside the first `total` samples.  Returns the rows, or 0 when no
-// map can be made.
-int encode_pcm_map(CUtensorMap* m, const float* pcm, int64_t total, int w = BLK) {
+// Offline spans land as their even and their odd 160-sample hop blocks in
+// two regions, one box each: the tensor views below take every other row of
+// the buffer, starting at row q (0 or 1), so a tile's hop blocks b, b + 2, ...
+// are consecutive z-rows of one view.
+constexpr int EO_BOX_ROWS = OFFLINE_SPAN_BLOCKS / 2;   // 17 hop blocks per region
+
+// The rows 2 z + q of the PCM as a 3-D tensor [z][40][w] whose element
+// (x, y, z) is pcm[160 q + 320 z + 4 y + x]: rows of w samples start at every
+// 16-byte boundary (for w = 164 the strides overlap on purpose), so one
+// 164 x 1 x 17 box lands the even or the odd hop blocks of any tile's span,
+// from the boundary at or before it, in their slots.  Rows are counted so
+// that every row of every start class lies inside the first `total` samples.
+// Returns the rows, or 0 when no map can be made.
+int encode_pcm_map(CUtensorMap* m, const float* pcm, int64_t total, int q, int w = BLK) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
-  const int64_t rows = total >= 4 * (HOP / 4 - 1) + w ? (total - 4 * (HOP / 4 - 1) - w) / HOP + 1 : 0;
+  const int64_t last = total - (int64_t)HOP * q - 4 * (HOP / 4 - 1) - w;   // start of the last full row, z = 0 based
+  const int64_t rows = last >= 0 ? last / (2 * HOP) + 1 : 0;
   if (!enc || (reinterpret_cast<uintptr_t>(pcm) & 15) || rows < 1 || rows >= INT32_MAX) return 0;
   cuuint64_t dims[3] = {(cuuint64_t)w, (cuuint64_t)(HOP / 4), (cuuint64_t)rows};
-  cuuint64_t strides[2] = {4 * sizeof(float), (cuuint64_t)HOP * sizeof(float)};
-  cuuint32_t box[3] = {(cuuint32_t)BLK, 1, (cuuint32_t)OFFLINE_SPAN_BLOCKS};
+  cuuint64_t strides[2] = {4 * sizeof(float), (cuuint64_t)(2 * HOP) * sizeof(float)};
+  cuuint32_t box[3] = {(cuuint32_t)BLK, 1, (cuuint32_t)EO_BOX_ROWS};
   cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(pcm), dims, strides, box, estr,
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(pcm + (int64_t)HOP * q), dims, strides, box,
+             estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS
              ? (int)rows
              : 0;
 }
 
-// The PCM as a 2-D tensor of 160-sample rows (contiguous) for one-box copies
-// of spans that start on a row; the box is 164 x 34 and its columns
+// The 160-sample rows 2 z + q of the PCM as a 2-D tensor [z][160] for the
+// copies of spans that start on a row; the box is 164 x 17 and its columns
 // 160..163 lie outside the tensor (zeros).  Returns the rows, or 0.
-int encode_pcm_rows(CUtensorMap* m, const float* pcm, int64_t total) {
+int encode_pcm_rows(CUtensorMap* m, const float* pcm, int64_t total, int q) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
-  const int64_t rows = total / HOP;
+  const int64_t all = total / HOP;                  // whole 160-sample rows of the buffer
+  const int64_t rows = all > q ? (all - q + 1) / 2 : 0;
   if (!enc || (reinterpret_cast<uintptr_t>(pcm) & 15) || rows < 1 || rows >= INT32_MAX) return 0;
   cuuint64_t dims[2] = {(cuuint64_t)HOP, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)HOP * sizeof(float)};
-  cuuint32_t box[2] = {(cuuint32_t)BLK, (cuuint32_t)OFFLINE_SPAN_BLOCKS};
+  cuuint64_t strides[1] = {(cuuint64_t)(2 * HOP) * sizeof(float)};
+  cuuint32_t box[2] = {(cuuint32_t)BLK, (cuuint32_t)EO_BOX_ROWS};
   cuuint32_t estr[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(pcm), dims, strides, box, estr,
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(pcm + (int64_t)HOP * q), dims, strides, box,
+             estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS
              ? (int)rows
@@ -189,11 +199,13 @@ struct logmel_plan {
   int ring_next = 0;
   Args mel{};               // filterbank fields copied into every launch
   bool default_mel = false; // structure equals the compiled default layout
-  // tensor map of the last offline PCM buffer (re-encoded when it changes)
-  CUtensorMap tmap{}, tmap_s{};
+  // tensor maps of the last offline PCM buffer (re-encoded when it changes)
+  CUtensorMap tmap[2]{}, tmap_s[2]{};
   const float* tmap_pcm = nullptr;
   int64_t tmap_len = -1;
-  int tmap_rows = 0, tmap_s_rows = 0;
+  int tmap_rows[2]{}, tmap_s_rows[2]{};
+  // bounded span waits (test hook; 0, 0 in normal operation)
+  int wait_polls = 0, tx_extra = 0;
   // tensor map of the last offline output buffer (full-tile row stores)
   CUtensorMap otmap{};
   const float* otmap_out = nullptr;
@@ -208,6 +220,11 @@ struct logmel_stream {
   int* d_carry_len = nullptr;
   std::vector<int64_t> total;    // samples received per stream
   std::vector<int> carry_len;    // host mirror of d_carry_len
+  // ragged pushes: per-stream chunk offsets, staged in a pinned ring and
+  // copied to the device ahead of the kernel (allocated on first use)
+  int64_t* d_push_off = nullptr;
+  PinnedSlot off_ring[RING];
+  int off_next = 0;
 };
 
 // ---------------------------------------------------------------------------
@@ -217,13 +234,20 @@ namespace {
 
 // New carry after a push whose frames were computed with the carry left in
 // place (pushes emitting more than one tile per stream): one CTA per stream.
+// push_off (ragged pushes): stream sl's chunk is chunks[push_off[sl] ..
+// push_off[sl + 1]); else len samples at chunks + sl * chunk_stride.
 __global__ void carry_update_kernel(float* carry, int* carry_len, const float* chunks,
-                                    int64_t chunk_stride, int64_t len, int stream_base) {
+                                    int64_t chunk_stride, int64_t len, int stream_base,
+                                    const int64_t* push_off) {
   __shared__ float buf[CARRY_CAP];
   const int sl = blockIdx.x;
   const int s = stream_base + sl;
   float* cs = carry + (int64_t)s * CARRY_CAP;
   const float* ch = chunks + (int64_t)sl * chunk_stride;
+  if (push_off != nullptr) {
+    ch = chunks + push_off[sl];
+    len = push_off[sl + 1] - push_off[sl];
+  }
   const int c = carry_len[s];            // read by every thread before the barrier
   const int64_t B = c + len;
   const int64_t nf = B >= NFFT ? (B - NFFT) / HOP + 1 : 0;
@@ -378,20 +402,24 @@ static void shape_launch(LaunchCfg& c, int span_blocks, int n_mels, int max_smem
 
 template <bool kDefault>
 static logmel_status setup_kernel(logmel_plan* p, int sms) {
-  const size_t mx = std::max(p->off.smem, p->str.smem);
-  if (cudaFuncSetAttribute(logmel_fused_kernel<kDefault, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)mx) != cudaSuccess ||
-      cudaFuncSetAttribute(logmel_fused_kernel<kDefault, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)mx) != cudaSuccess)
+  if (cudaFuncSetAttribute(logmel_fused_kernel<kDefault, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)p->off.smem) != cudaSuccess ||
+      cudaFuncSetAttribute(logmel_fused_kernel<kDefault, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)p->off.smem) != cudaSuccess ||
+      cudaFuncSetAttribute(logmel_fused_kernel<kDefault, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)p->str.smem) != cudaSuccess)
     return LOGMEL_ERR_CUDA;
-  for (LaunchCfg* c : {&p->off, &p->str}) {
-    int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, logmel_fused_kernel<kDefault, false>,
-                                                      c->groups * GROUP_THREADS, c->smem) != cudaSuccess ||
-        occ < 1)
-      return LOGMEL_ERR_CUDA;
-    c->max_ctas = sms * occ;
-  }
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, logmel_fused_kernel<kDefault, false, false>,
+                                                    p->off.groups * GROUP_THREADS, p->off.smem) != cudaSuccess ||
+      occ < 1)
+    return LOGMEL_ERR_CUDA;
+  p->off.max_ctas = sms * occ;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, logmel_fused_kernel<kDefault, false, true>,
+                                                    p->str.groups * GROUP_THREADS, p->str.smem) != cudaSuccess ||
+      occ < 1)
+    return LOGMEL_ERR_CUDA;
+  p->str.max_ctas = sms * occ;
   return LOGMEL_OK;
 }
 
@@ -407,7 +435,10 @@ static cudaError_t launch(const logmel_plan* p, Args& a, int64_t tiles, cudaStre
     }
   }
   a.tables = p->d_tables;
+  a.wait_polls = p->wait_polls;
+  a.tx_extra = p->tx_extra;
   a.span_blocks = c.span_blocks;
+  a.eo_off = eo_off_for(c.span_blocks);
   a.group_bytes = c.group_bytes;
   a.ybuf_bytes = c.ybuf_bytes;
   a.bulk_store = p->default_mel && (reinterpret_cast<uintptr_t>(a.out) & 15) == 0;
@@ -418,12 +449,15 @@ static cudaError_t launch(const logmel_plan* p, Args& a, int64_t tiles, cudaStre
   std::memcpy(a.warp_band, p->mel.warp_band, sizeof a.warp_band);
   const int grid = (int)std::min<int64_t>((tiles + c.groups - 1) / c.groups, c.max_ctas);
   const int block = c.groups * GROUP_THREADS;
-  if (p->default_mel) {
-    if (odd) logmel_fused_kernel<true, true><<<grid, block, c.smem, s>>>(a);
-    else logmel_fused_kernel<true, false><<<grid, block, c.smem, s>>>(a);
+  if (a.mode == 1) {
+    if (p->default_mel) logmel_fused_kernel<true, false, true><<<grid, block, c.smem, s>>>(a);
+    else logmel_fused_kernel<false, false, true><<<grid, block, c.smem, s>>>(a);
+  } else if (p->default_mel) {
+    if (odd) logmel_fused_kernel<true, true, false><<<grid, block, c.smem, s>>>(a);
+    else logmel_fused_kernel<true, false, false><<<grid, block, c.smem, s>>>(a);
   } else {
-    if (odd) logmel_fused_kernel<false, true><<<grid, block, c.smem, s>>>(a);
-    else logmel_fused_kernel<false, false><<<grid, block, c.smem, s>>>(a);
+    if (odd) logmel_fused_kernel<false, true, false><<<grid, block, c.smem, s>>>(a);
+    else logmel_fused_kernel<false, false, false><<<grid, block, c.smem, s>>>(a);
   }
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -648,13 +682,17 @@ logmel_status logmel_compute(logmel_plan* p, const float* pcm, const int64_t* of
   if (pcm != p->tmap_pcm || total != p->tmap_len) {
     p->tmap_pcm = pcm;
     p->tmap_len = total;
-    p->tmap_rows = encode_pcm_rows(&p->tmap, pcm, total);
-    p->tmap_s_rows = encode_pcm_map(&p->tmap_s, pcm, total, BLK);
+    for (int q = 0; q < 2; ++q) {
+      p->tmap_rows[q] = encode_pcm_rows(&p->tmap[q], pcm, total, q);
+      p->tmap_s_rows[q] = encode_pcm_map(&p->tmap_s[q], pcm, total, q, BLK);
+    }
   }
-  a.tmap = p->tmap;
-  a.tmap_rows = p->tmap_rows;
-  a.tmap_s = p->tmap_s;
-  a.tmap_s_rows = p->tmap_s_rows;
+  for (int q = 0; q < 2; ++q) {
+    a.tmap[q] = p->tmap[q];
+    a.tmap_rows[q] = p->tmap_rows[q];
+    a.tmap_s[q] = p->tmap_s[q];
+    a.tmap_s_rows[q] = p->tmap_s_rows[q];
+  }
   if (p->default_mel) {
     if (out != p->otmap_out || frames != p->otmap_len) {
       p->otmap_out = out;
@@ -705,6 +743,11 @@ void logmel_stream_destroy(logmel_stream* st) {
   cudaDeviceSynchronize();
   cudaFree(st->d_carry);
   cudaFree(st->d_carry_len);
+  cudaFree(st->d_push_off);
+  for (int i = 0; i < RING; ++i) {
+    if (st->off_ring[i].host) cudaFreeHost(st->off_ring[i].host);
+    if (st->off_ring[i].done) cudaEventDestroy(st->off_ring[i].done);
+  }
   delete st;
 }
 
@@ -720,24 +763,83 @@ int64_t logmel_stream_max_frames(const logmel_stream* st, int64_t len) {
   return mx;
 }
 
+// Pinned staging of a ragged push's chunk offsets and their device copy.
+static logmel_status stage_push_offsets(logmel_stream* st, const int64_t* off, int count,
+                                        cudaStream_t s, const int64_t** d_off) {
+  const size_t bytes = sizeof(int64_t) * ((size_t)st->n_streams + 1);
+  if (!st->d_push_off) {
+    if (cudaMalloc(&st->d_push_off, bytes) != cudaSuccess) {
+      st->d_push_off = nullptr;
+      return LOGMEL_ERR_OOM;
+    }
+    for (int i = 0; i < RING; ++i) {
+      if (cudaHostAlloc(&st->off_ring[i].host, bytes, cudaHostAllocDefault) != cudaSuccess) {
+        st->off_ring[i].host = nullptr;
+        return LOGMEL_ERR_OOM;
+      }
+      CK(cudaEventCreateWithFlags(&st->off_ring[i].done, cudaEventDisableTiming));
+    }
+  }
+  PinnedSlot& slot = st->off_ring[st->off_next];
+  st->off_next = (st->off_next + 1) % RING;
+  if (slot.used) CK(cudaEventSynchronize(slot.done));
+  std::memcpy(slot.host, off, sizeof(int64_t) * ((size_t)count + 1));
+  CK(cudaMemcpyAsync(st->d_push_off, slot.host, sizeof(int64_t) * ((size_t)count + 1),
+                     cudaMemcpyHostToDevice, s));
+  CK(cudaEventRecord(slot.done, s));
+  slot.used = true;
+  *d_off = st->d_push_off;
+  return LOGMEL_OK;
+}
+
+// One push to streams base .. base + count - 1: either every stream takes
+// len samples at chunks + i * chunk_stride (h_off == nullptr), or stream
+// base + i takes chunks[h_off[i] .. h_off[i + 1]) (h_off: host, count + 1
+// entries, non-decreasing).
+int64_t logmel_stream_max_frames_ragged(const logmel_stream* st, const int64_t* off) {
+  if (!st || !off || off[0] < 0) return -1;
+  int64_t mx = 0;
+  for (int s = 0; s < st->n_streams; ++s) {
+    if (off[s + 1] < off[s]) return -1;
+    mx = std::max(mx, frames_of(st->carry_len[s] + (off[s + 1] - off[s])));
+  }
+  return mx;
+}
+
 static logmel_status push_impl(logmel_stream* st, int base, int count, const float* chunks,
                                int64_t chunk_stride, int64_t len, float* out, int64_t cap,
-                               int64_t* n_out, void* stream) {
+                               int64_t* n_out, void* stream, const int64_t* h_off = nullptr) {
   logmel_plan* p = st->plan;
-  if (len < 0 || cap < 0 || !n_out) return LOGMEL_ERR_INVALID_ARG;
+  if (cap < 0 || !n_out) return LOGMEL_ERR_INVALID_ARG;
+  auto len_of = [&](int i) { return h_off ? h_off[i + 1] - h_off[i] : len; };
+  if (h_off) {
+    if (h_off[0] < 0) return LOGMEL_ERR_INVALID_ARG;
+    len = 0;
+    for (int i = 0; i < count; ++i) {
+      if (h_off[i + 1] < h_off[i]) return LOGMEL_ERR_INVALID_ARG;
+      len = std::max(len, h_off[i + 1] - h_off[i]);
+    }
+    if (h_off[count] >= (int64_t)INT32_MAX * 64) return LOGMEL_ERR_INPUT_TOO_LONG;
+  }
+  if (len < 0) return LOGMEL_ERR_INVALID_ARG;
   if (len > (int64_t)INT32_MAX / 2) return LOGMEL_ERR_INPUT_TOO_LONG;
   int64_t max_n = 0;
-  for (int i = 0; i < count; ++i) max_n = std::max(max_n, frames_of(st->carry_len[base + i] + len));
+  for (int i = 0; i < count; ++i) max_n = std::max(max_n, frames_of(st->carry_len[base + i] + len_of(i)));
   if (max_n > cap) return LOGMEL_ERR_INVALID_ARG;
   if (len > 0 && !chunks) return LOGMEL_ERR_INVALID_ARG;
   if (max_n > 0 && !out) return LOGMEL_ERR_INVALID_ARG;
-  if (count > 1 && chunk_stride < len) return LOGMEL_ERR_INVALID_ARG;
+  if (!h_off && count > 1 && chunk_stride < len) return LOGMEL_ERR_INVALID_ARG;
   const int spt = max_n <= TILE / 4 ? 4 : (max_n <= TILE / 2 ? 2 : 1);
   const int64_t tps = max_n <= TILE ? 1 : (max_n + TILE - 1) / TILE;
   const int64_t tiles = (int64_t)((count + spt - 1) / spt) * tps;
   if (tiles >= INT32_MAX || (int64_t)count * cap >= INT32_MAX) return LOGMEL_ERR_INPUT_TOO_LONG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (len > 0) {
+    const int64_t* d_off = nullptr;
+    if (h_off) {
+      const logmel_status so = stage_push_offsets(st, h_off, count, s, &d_off);
+      if (so != LOGMEL_OK) return so;
+    }
     Args a{};
     a.out = out;
     a.status = p->d_status;
@@ -749,6 +851,7 @@ static logmel_status push_impl(logmel_stream* st, int base, int count, const flo
     a.chunks = chunks;
     a.chunk_stride = chunk_stride;
     a.push_len = len;
+    a.push_off = d_off;
     a.stream_base = base;
     a.n_push_streams = count;
     a.spt = spt;
@@ -758,17 +861,17 @@ static logmel_status push_impl(logmel_stream* st, int base, int count, const flo
     if (launch(p, a, tiles, s) != cudaSuccess) return LOGMEL_ERR_CUDA;
     if (tps > 1) {
       carry_update_kernel<<<count, 128, 0, s>>>(st->d_carry, st->d_carry_len, chunks, chunk_stride,
-                                                len, base);
+                                                len, base, d_off);
       CK(cudaGetLastError());
     }
   }
   for (int i = 0; i < count; ++i) {
     const int id = base + i;
-    const int64_t B = st->carry_len[id] + len;
+    const int64_t B = st->carry_len[id] + len_of(i);
     const int64_t n = frames_of(B);
     n_out[i] = n;
     st->carry_len[id] = (int)(B - n * HOP);
-    st->total[id] += len;
+    st->total[id] += len_of(i);
   }
   return LOGMEL_OK;
 }
@@ -784,6 +887,13 @@ logmel_status logmel_stream_push_batch(logmel_stream* st, const float* chunks, i
                                        void* stream) {
   if (!st) return LOGMEL_ERR_INVALID_ARG;
   return push_impl(st, 0, st->n_streams, chunks, stride, len, out, cap, n_out, stream);
+}
+
+logmel_status logmel_stream_push_batch_ragged(logmel_stream* st, const float* chunks,
+                                              const int64_t* chunk_offsets, float* out, int64_t cap,
+                                              int64_t* n_out, void* stream) {
+  if (!st || !chunk_offsets) return LOGMEL_ERR_INVALID_ARG;
+  return push_impl(st, 0, st->n_streams, chunks, 0, 0, out, cap, n_out, stream, chunk_offsets);
 }
 
 struct StateHeader {
@@ -865,6 +975,14 @@ logmel_status logmel_stream_reset(logmel_stream* st, int id, void* stream) {
     st->total[id] = 0;
     st->carry_len[id] = 0;
   }
+  return LOGMEL_OK;
+}
+
+logmel_status logmel_plan_set_wait_test(logmel_plan* p, int extra_tx_bytes, int poll_limit) {
+  if (!p || extra_tx_bytes < 0 || extra_tx_bytes > (1 << 20) || extra_tx_bytes % 16 || poll_limit < 0)
+    return LOGMEL_ERR_INVALID_ARG;
+  p->tx_extra = extra_tx_bytes;
+  p->wait_polls = poll_limit;
   return LOGMEL_OK;
 }
 
@@ -1040,8 +1158,10 @@ extern "C" logmel_status logmel_compute_noalloc(const float* pcm, const int64_t*
   a.status = status;
   a.mode = 0;
   // the PCM as a tensor for one-box tile copies, as in logmel_compute
-  a.tmap_rows = encode_pcm_rows(&a.tmap, pcm, off[n_utt]);
-  a.tmap_s_rows = encode_pcm_map(&a.tmap_s, pcm, off[n_utt], BLK);
+  for (int q = 0; q < 2; ++q) {
+    a.tmap_rows[q] = encode_pcm_rows(&a.tmap[q], pcm, off[n_utt], q);
+    a.tmap_s_rows[q] = encode_pcm_map(&a.tmap_s[q], pcm, off[n_utt], q, BLK);
+  }
   a.otmap_rows = encode_out_map(&a.otmap, out, frames, d.plan.n_mels);
   a.num_tiles = (int)tiles;
   a.n_mels = d.plan.n_mels;

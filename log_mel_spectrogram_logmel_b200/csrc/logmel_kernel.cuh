@@ -5,17 +5,21 @@
 // samples -> symmetric Hamming window -> real DFT (201 bins) -> |X|^2 ->
 // 128 triangular mel filters -> ln(max(., 1e-10)).
 //
-// Structure (one persistent kernel; tile groups of 160 threads, up to three
-// per CTA, each working through tiles of 32 frames; frame slots d and d + 16
-// form the pair carried by one thread):
+// Structure (one persistent kernel per mode -- offline batch or streaming
+// push; tile groups of 160 threads, up to three per CTA, each working
+// through tiles of 32 frames; adjacent frame slots 2p and 2p + 1 form the
+// pair carried by one thread):
 //   stage   each tile's overlapping sample span is copied from HBM once into
 //           shared memory by the bulk-copy (TMA) engine, as 34 hop blocks of
 //           160 samples in 164-float slots, from the 16-byte boundary at or
 //           before the span (the slots then hold their samples from that
-//           shift): one 2-D tensor copy when the span starts on a 160-sample
-//           row, else one 3-D tensor copy over overlapping rows, else one
-//           bulk copy per hop block, else cp.async; a half-warp reads 8 frame
-//           pairs x 2 roles, so pass A's strided reads are conflict-free
+//           shift); even and odd hop blocks go to two separate regions, so
+//           that frames 2p and 2p + 1 (blocks 2p .. 2p + 3) sit at the same
+//           bank offsets: two tensor copies (one per region) when the span
+//           starts on a 160-sample row or on any 16-byte boundary, else one
+//           bulk copy per hop block, else cp.async; frame 2p + 1 reuses 12 of
+//           frame 2p's 20 sample pairs (28 loads per frame pair, not 40), and
+//           a half-warp reads 8 frame pairs x 2 roles without conflicts
 //   pass A  real FFT-400 as a complex FFT-200 of z[m] = x[2m] + i x[2m+1]
 //           (window applied on load), Cooley-Tukey 200 = 20 x 10: ten
 //           20-point DFTs per frame (prime-factor 4 x 5, no inner twiddles),
@@ -105,23 +109,26 @@ struct TileDesc {
 };
 
 struct Args {
-  // offline: two tensor views of the PCM for one-box tile copies.
-  // tmap: rows of 160 samples (2-D, contiguous rows); a 164 x 34 box lands a
-  // span that starts on a row in its hop-block slots, columns 160..163 lying
-  // outside the tensor (zeros, not read).  tmap_s: a 3-D tensor whose
-  // element (x, y, z) is pcm[160 z + 4 y + x], rows of 164 samples starting
-  // at every 16-byte boundary (overlapping strides); a 164 x 1 x 34 box lands
-  // any other span from the boundary at or before it, shifted by its offset.
-  CUtensorMap tmap;
-  CUtensorMap tmap_s;
+  // offline: tensor views of the PCM for the tile copies, one per parity q
+  // of the 160-sample rows (row 2 z + q of the buffer is z-row z of view q),
+  // so that one box lands every other hop block of a span in one region.
+  // tmap[q]: element (x, z) is pcm[160 q + 320 z + x], x < 160; a 164 x 17
+  // box lands the even (or odd) hop blocks of a span that starts on a row,
+  // columns 160..163 lying outside the tensor (zeros, not read).
+  // tmap_s[q]: element (x, y, z) is pcm[160 q + 320 z + 4 y + x], rows of 164
+  // samples starting at every 16-byte boundary (overlapping strides); a
+  // 164 x 1 x 17 box lands those of any other span from the boundary at or
+  // before it, shifted by its offset.
+  CUtensorMap tmap[2];
+  CUtensorMap tmap_s[2];
   // offline: the output as a 2-D tensor [rows][n_mels]; an
   // orow_floats(n_mels) x 32 box stores one full tile's staged rows (the pad
   // columns fall outside the tensor)
   CUtensorMap otmap;
-  int tmap_rows;        // rows of tmap (0: no tensor map)
-  int tmap_s_rows;      // rows (z extent) of tmap_s (0: none)
+  int tmap_rows[2];     // z extent of tmap[q] (0: no tensor map)
+  int tmap_s_rows[2];   // z extent of tmap_s[q] (0: none)
   int otmap_rows;       // rows of the output tensor (0: no tensor map)
-  int pad_tm_[1];
+  int eo_off;           // floats from the even-block region to the odd-block region
   const Tables* tables;
   TileDesc* tiles;      // offline: per-tile descriptors (written by the kernel's prologue)
   float* out;
@@ -147,12 +154,20 @@ struct Args {
   const float* chunks;
   int64_t chunk_stride;
   int64_t push_len;
+  const int64_t* push_off;     // ragged push (device, [n_push_streams + 1]): stream sl's chunk is
+                               // chunks[push_off[sl] .. push_off[sl + 1]); nullptr: every stream
+                               // pushes push_len samples from chunks + sl * chunk_stride
   int stream_base;
   int n_push_streams;
   int spt;                     // streams per tile (1, 2, 4)
   int tps;                     // tiles per stream
   int update_carry;            // 1: this kernel writes the new carries
   int64_t out_cap;             // output rows per stream
+  // bounded waits: polls before a span copy counts as lost (0: 65536, about
+  // 65 ms), and bytes added to each tile's expected copy bytes (0; a test
+  // sets them to make the wait run out while every real copy still lands)
+  int wait_polls;
+  int tx_extra;
   // filterbank (per plan): weights / 4 (the real split yields |2 X|^2), and
   // for the generic (non-default) layout the band structure
   float mel_w[MAX_WEIGHTS];
@@ -257,22 +272,26 @@ __device__ __forceinline__ void dft10(cx (&x)[10]) {
 }
 
 // Pass A input: z[m1] = windowed (x[n], x[n + 1]) of the pair's two frames,
-// n = 20 m1 + 2 m2, read from the staged span (kOdd: the samples sit at an
-// odd float offset, so each pair takes two 4-byte loads).
+// n = 20 m1 + 2 m2, read from the staged span: sample n of frame A sits at
+// pa[n / 160] + (n mod 160), of frame B at pb[n / 160] + (n mod 160), where
+// pa[j], pb[j] are the frames' hop-block slots (offset by 2 m2 and the
+// shift).  Offline pairs are adjacent frames of one utterance, so pb[0] and
+// pb[1] are the same slots as pa[1] and pa[2] and their loads are shared
+// (kOdd: the samples sit at an odd float offset, so each pair takes two
+// 4-byte loads).
 template <bool kOdd>
-__device__ __forceinline__ void window_load(cx (&z)[N1], const float* sa, const float* sb, const Tables& tab,
-                                            int m2) {
+__device__ __forceinline__ float2 ld_pair(const float* q) {
+  if constexpr (kOdd) return make_float2(q[0], q[1]);
+  else return *reinterpret_cast<const float2*>(q);
+}
+template <bool kOdd>
+__device__ __forceinline__ void window_load(cx (&z)[N1], const float* const (&pa)[3], const float* const (&pb)[3],
+                                            const Tables& tab, int m2) {
 #pragma unroll
   for (int m1 = 0; m1 < N1; ++m1) {
-    const int off = BLK * (m1 / 8) + 20 * (m1 % 8);   // sample n = 20 m1 + 2 m2
-    float2 xa, xb;
-    if constexpr (kOdd) {
-      xa = make_float2(sa[off], sa[off + 1]);
-      xb = make_float2(sb[off], sb[off + 1]);
-    } else {
-      xa = *reinterpret_cast<const float2*>(sa + off);
-      xb = *reinterpret_cast<const float2*>(sb + off);
-    }
+    const int off = 20 * (m1 % 8);   // sample n = 20 m1 + 2 m2 in hop block m1 / 8
+    const float2 xa = ld_pair<kOdd>(pa[m1 / 8] + off);
+    const float2 xb = ld_pair<kOdd>(pb[m1 / 8] + off);
     const float4 w4 = *reinterpret_cast<const float4*>(&tab.win[m2][m1 & ~1]);
     const float2 w = (m1 & 1) ? make_float2(w4.z, w4.w) : make_float2(w4.x, w4.y);
     z[m1].re = make_float2(xa.x * w.x, xb.x * w.x);
@@ -286,7 +305,7 @@ __device__ __forceinline__ cx sel(bool p, const cx& a, const cx& b) {
 
 // ---------------------------------------------------------------------------
 // shared memory layout: [tables] then, per tile group of 160 threads,
-// [control block x 2][pass buffer][span region]
+// [control block x 2][pass buffer][span region: even hop blocks | odd hop blocks]
 //   control      groups and per-slot rows of the current and the next tile
 //   pass buffer  pass-A output (float4 per complex pair); after pass B has
 //                read it, the power rows [199 bins][32 frame columns] and
@@ -296,7 +315,9 @@ __device__ __forceinline__ cx sel(bool p, const cx& a, const cx& b) {
 //                store)
 // A CTA runs several independent tile groups (named barriers per group), so
 // the tables are held once per CTA.  Offline tiles need 34 hop blocks of
-// span, streaming tiles with four groups 40.
+// span, streaming tiles with four groups 40.  Hop block b of a span sits in
+// the even region at (b / 2) * BLK, or in the odd region (which starts on a
+// 128-byte boundary) at eo_off + (b / 2) * BLK.
 // ---------------------------------------------------------------------------
 constexpr int GROUP_THREADS = 160;
 constexpr int MAX_TILE_GROUPS = 3;
@@ -306,13 +327,14 @@ struct __align__(16) Ctl {
   int ngroups;
   int nslots;
   int tma;                  // staging: kind | (shift << 2).  kind 0: cp.async; 1: bulk copies
-                            // per hop block; 2: one tensor copy (both wait on bar).  shift
-                            // (0..3): the slots hold their samples from position shift
-                            // (copies start at the 16-byte boundary before the span)
+                            // per hop block; 2: two tensor copies, one per block region
+                            // (both kinds wait on bar).  shift (0..3): the slots hold their
+                            // samples from position shift (copies start at the 16-byte
+                            // boundary before the span)
   int bar_parity;           // phase of bar to wait for
   int copy_ok;              // verdict on the bulk copies (0: a thread's bounded wait gave up)
-  int tmap_row;             // tensor copy: row and start class of the box (see Args::tmap)
-  int tmap_y;
+  int tmap_row;             // tensor copies: the span's first 160-sample row of the buffer
+  int tmap_y;               // and its start class (-1: on a row; see Args::tmap)
   TileDesc pending;         // offline: the descriptor of the group's tile after next
   int early;                // 1: the first tile's copy was issued before the prologue's barrier
 };
@@ -342,19 +364,33 @@ __host__ __device__ constexpr int ybuf_bytes_for(int n_mels) {
 }
 static_assert(PROWS_FLOATS * 4 % 128 == 0, "output rows start 128-byte aligned");
 static_assert(YBUF_BYTES % 128 == 0 && CTL_BYTES % 128 == 0 && TAB_BYTES % 128 == 0, "128-byte aligned regions");
+// floats from the even-block region to the odd-block region (128-byte aligned)
+__host__ __device__ constexpr int eo_off_for(int span_blocks) {
+  return ((span_blocks + 1) / 2 * BLK + 31) / 32 * 32;
+}
+__host__ __device__ constexpr int span_floats_for(int span_blocks) {
+  return eo_off_for(span_blocks) + span_blocks / 2 * BLK;
+}
 __host__ __device__ constexpr int group_bytes_for(int span_blocks, int n_mels) {
-  return (2 * CTL_BYTES + ybuf_bytes_for(n_mels) + span_blocks * BLK * 4 + 127) / 128 * 128;
+  return (2 * CTL_BYTES + ybuf_bytes_for(n_mels) + span_floats_for(span_blocks) * 4 + 127) / 128 * 128;
+}
+// the slot of hop block b in the span region
+__device__ __forceinline__ float* blk_addr(float* span, int eo, int b) {
+  return span + ((b & 1) ? eo : 0) + (b >> 1) * BLK;
+}
+__device__ __forceinline__ const float* blk_addr(const float* span, int eo, int b) {
+  return span + ((b & 1) ? eo : 0) + (b >> 1) * BLK;
 }
 // Three offline tile groups of the default 128-band layout must fit in the
 // 232,448 bytes of shared memory an sm_100 CTA may opt into (15 warps per SM).
 static_assert(TAB_BYTES + MAX_TILE_GROUPS * group_bytes_for(OFFLINE_SPAN_BLOCKS, 128) <= 232448,
               "three default tile groups per CTA");
 
-// Power-row column of frame slot f for a bin of parity par: the frames d and
-// d + 16 of a pair sit in columns 2d and 2d + 1, and odd bins swap the two
-// column halves (the two roles of a warp write rows of opposite parity, so
-// their 8-byte pair stores hit distinct banks).
-__device__ __forceinline__ int pcol(int f, int par) { return (2 * (f & 15) + (f >> 4)) ^ (16 * par); }
+// Power-row column of frame slot f for a bin of parity par: the frames 2p
+// and 2p + 1 of a pair sit in columns 2p and 2p + 1, and odd bins swap the
+// two column halves (the two roles of a warp write rows of opposite parity,
+// so their 8-byte pair stores hit distinct banks).
+__device__ __forceinline__ int pcol(int f, int par) { return f ^ (16 * par); }
 
 __device__ __forceinline__ void group_sync(int g) {
   asm volatile("bar.sync %0, %1;" ::"r"(g + 1), "r"(GROUP_THREADS) : "memory");
@@ -535,11 +571,16 @@ __device__ void setup_offline(Ctl& S, const Args& a, const TileDesc& t, const fl
   const bool shift_ok = odd_ok || !(r & 1);
   const int yk = (int)(a0 - row * HOP) / 4;   // start class: 4 yk floats into a 160-sample row
   const bool on_row = r == 0 && yk == 0;
-  const int map_rows = on_row ? a.tmap_rows : a.tmap_s_rows;
-  if (map_rows > 0 && shift_ok && a0 >= 0 && row + nb <= map_rows && (smem_addr(span) & 127) == 0) {
+  // even hop blocks: buffer rows row, row + 2, ... = z-rows from row / 2 of
+  // the view of parity row & 1; odd ones: from (row + 1) / 2 of the other
+  const int* map_rows = on_row ? a.tmap_rows : a.tmap_s_rows;
+  const int qe = (int)(row & 1), ne = (nb + 1) / 2, no = nb / 2;
+  const bool fits = a0 >= 0 && map_rows[qe] > 0 && (row >> 1) + ne <= map_rows[qe] &&
+                    (no == 0 || (map_rows[qe ^ 1] > 0 && ((row + 1) >> 1) + no <= map_rows[qe ^ 1]));
+  if (fits && shift_ok && (smem_addr(span) & 127) == 0) {
     S.tma = 2 | (r << 2);
     S.tmap_row = (int)row;
-    S.tmap_y = on_row ? -1 : yk;   // -1: the 2-D row map
+    S.tmap_y = on_row ? -1 : yk;   // -1: the row views
   } else if ((reinterpret_cast<uintptr_t>(g.src0) & 15) == 0) {
     S.tma = 1;
   } else if (shift_ok && (reinterpret_cast<uintptr_t>(g.src0) & 3) == 0 && g.src0 - r >= a.pcm &&
@@ -558,8 +599,15 @@ __device__ void setup_stream(Ctl& S, const Args& a, int tile) {
     const int sl = sg * a.spt + j;
     if (sl >= a.n_push_streams) break;
     const int s = a.stream_base + sl;
+    int64_t len = a.push_len;
+    const float* chunk = a.chunks + (int64_t)sl * a.chunk_stride;
+    if (a.push_off != nullptr) {
+      chunk = a.chunks + a.push_off[sl];
+      len = a.push_off[sl + 1] - a.push_off[sl];
+      if (len == 0) continue;   // nothing arrives: the stream's state stays as it is
+    }
     const int c = a.carry_len[s];
-    const int64_t B = c + a.push_len;
+    const int64_t B = c + len;
     const int64_t n = B >= NFFT ? (B - NFFT) / HOP + 1 : 0;
     const int64_t f0 = (int64_t)st * TILE;
     const int cnt = (int)max64(0, min64(TILE / a.spt, n - f0));
@@ -567,7 +615,7 @@ __device__ void setup_stream(Ctl& S, const Args& a, int tile) {
     if (cnt == 0 && !owner) continue;
     Group& g = S.groups[ng];
     g.src0 = a.carry + (int64_t)s * CARRY_CAP;
-    g.src1 = a.chunks + (int64_t)sl * a.chunk_stride;
+    g.src1 = chunk;
     g.len0 = c;
     g.start = f0 * HOP;
     // stage the frames' samples; a group with no frames (a push too short
@@ -604,61 +652,70 @@ __device__ void setup_stream(Ctl& S, const Args& a, int tile) {
 // whose pass-B share is the lightest).
 constexpr int COPY_TID = 128;
 
+template <bool kStream>
 __device__ __forceinline__ void stage_tile(Ctl& S, float* span, int tid, const Args& a) {
-  if ((S.tma & 3) == 2) {   // one 164 x 1 x 34 tensor box per tile
+  const int eo = a.eo_off;
+  if (!kStream && (S.tma & 3) == 2) {   // two 164 x 17 tensor boxes: the even and the odd hop blocks
     if (tid == COPY_TID) {
-      mbar_expect_tx(&S.bar, (unsigned)(BLK * OFFLINE_SPAN_BLOCKS * 4));
-      if (S.tmap_y < 0) tensor_load_2d(span, &a.tmap, 0, S.tmap_row, &S.bar);
-      else tensor_load_3d(span, &a.tmap_s, 0, S.tmap_y, S.tmap_row, &S.bar);
+      mbar_expect_tx(&S.bar, (unsigned)(BLK * OFFLINE_SPAN_BLOCKS * 4 + a.tx_extra));
+      const int R = S.tmap_row, q = R & 1;
+      if (S.tmap_y < 0) {
+        tensor_load_2d(span, &a.tmap[q], 0, R >> 1, &S.bar);
+        tensor_load_2d(span + eo, &a.tmap[q ^ 1], 0, (R + 1) >> 1, &S.bar);
+      } else {
+        tensor_load_3d(span, &a.tmap_s[q], 0, S.tmap_y, R >> 1, &S.bar);
+        tensor_load_3d(span + eo, &a.tmap_s[q ^ 1], 0, S.tmap_y, (R + 1) >> 1, &S.bar);
+      }
     }
     return;
   }
-  if (S.tma >= 4) {   // shifted: 164 floats per hop block from the 16-byte boundary before it
+  if (!kStream && S.tma >= 4) {   // shifted: 164 floats per hop block from the 16-byte boundary before it
     const Group& g = S.groups[0];
     if (tid >= COPY_TID && tid < COPY_TID + 32) {
       const int l = tid - COPY_TID;
       const int r = S.tma >> 2;
       const int nb = (g.nstage + HOP - 1) / HOP;
       const int total = (g.nstage + r + 3) & ~3;   // floats from src0 - r, a multiple of 4
-      if (l == 0) mbar_expect_tx(&S.bar, 4u * (unsigned)(BLK * (nb - 1) + (total - HOP * (nb - 1))));
+      if (l == 0) mbar_expect_tx(&S.bar, 4u * (unsigned)(BLK * (nb - 1) + (total - HOP * (nb - 1))) + a.tx_extra);
       __syncwarp();
       for (int b = l; b < nb; b += 32) {
         const int len = min(BLK, total - b * HOP);   // 164, the last block what is left
-        bulk_load(span + b * BLK, g.src0 - r + b * HOP, (unsigned)len * 4u, &S.bar);
+        bulk_load(blk_addr(span, eo, b), g.src0 - r + b * HOP, (unsigned)len * 4u, &S.bar);
       }
     }
     return;
   }
-  if (S.tma) {   // one bulk copy per hop block (640 B; the last one 320 B)
+  if (!kStream && S.tma) {   // one bulk copy per hop block (640 B; the last one 320 B)
     const Group& g = S.groups[0];
     if (tid >= COPY_TID && tid < COPY_TID + 32) {
       const int l = tid - COPY_TID;
       const int nb = (g.nstage + HOP - 1) / HOP;
-      if (l == 0) mbar_expect_tx(&S.bar, (unsigned)g.nstage * 4u);
+      if (l == 0) mbar_expect_tx(&S.bar, (unsigned)g.nstage * 4u + a.tx_extra);
       __syncwarp();
       for (int b = l; b < nb; b += 32) {
         const int len = min(HOP, g.nstage - b * HOP);
-        bulk_load(span + (g.block0 + b) * BLK, g.src0 + b * HOP, (unsigned)len * 4u, &S.bar);
+        bulk_load(blk_addr(span, eo, g.block0 + b), g.src0 + b * HOP, (unsigned)len * 4u, &S.bar);
       }
     }
     return;
   }
   for (int gi = 0; gi < S.ngroups; ++gi) {
     const Group& g = S.groups[gi];
-    float* dst = span + g.block0 * BLK;
     const float* base = g.src0 + g.start;
     const int n = g.nstage;   // <= 31 * 160 + 400 (frames) or < 400 (carry only)
     if (g.src1 == nullptr && (reinterpret_cast<uintptr_t>(base) & 7) == 0) {
-      const int hb = (2 * tid) >= HOP;                 // 2 tid + 320 q sits in block 2 q + hb
-      float* d0 = dst + hb * BLK + 2 * tid - hb * HOP;
+      // offline (block0 = 0): 2 tid + 320 q sits in hop block 2 q + hb,
+      // the q-th slot of the even (hb = 0) or the odd (hb = 1) region
+      const int hb = (2 * tid) >= HOP;
+      float* d0 = span + (hb ? eo : 0) + 2 * tid - hb * HOP;
       const float* s0 = base + 2 * tid;
 #pragma unroll
       for (int q = 0; q < (31 * HOP + NFFT + 2 * HOP - 1) / (2 * HOP); ++q)
-        if (2 * tid + 2 * HOP * q < n) cp_async8(d0 + 2 * BLK * q, s0 + 2 * HOP * q);
+        if (2 * tid + 2 * HOP * q < n) cp_async8(d0 + BLK * q, s0 + 2 * HOP * q);
     } else if (g.src1 == nullptr) {
 #pragma unroll
       for (int q = 0; q < (31 * HOP + NFFT + HOP - 1) / HOP; ++q)
-        if (tid + HOP * q < n) cp_async4(dst + BLK * q + tid, base + tid + HOP * q);
+        if (tid + HOP * q < n) cp_async4(blk_addr(span, eo, g.block0 + q) + tid, base + tid + HOP * q);
     } else {
       // streaming (carry ++ chunk): a push stages far fewer samples than the
       // span holds, so the loop runs over the staged hop blocks only
@@ -666,7 +723,7 @@ __device__ __forceinline__ void stage_tile(Ctl& S, float* span, int tid, const A
       for (int q = 0; HOP * q < n; ++q) {
         const int64_t pos = g.start + tid + HOP * q;
         if (tid + HOP * q < n)
-          cp_async4(dst + BLK * q + tid, pos < g.len0 ? g.src0 + pos : g.src1 + (pos - g.len0));
+          cp_async4(blk_addr(span, eo, g.block0 + q) + tid, pos < g.len0 ? g.src0 + pos : g.src1 + (pos - g.len0));
       }
     }
   }
@@ -789,18 +846,39 @@ __device__ __forceinline__ void split_power(const Tables& tab, const cx& zk, con
   pm = fma2(qi, qi, mul2(qr, qr));
 }
 
-// Pass A for one thread (frame pair d, role m2): windowed loads, 20-point
-// DFT over m1, twiddle; then, once the previous tile has released the pass
-// buffer (warp 0 waits for its row copies; group barrier), the stores of
-// the 20 outputs.  Returns the group's copy verdict (false: stop).
-template <bool kOdd>
-__device__ __forceinline__ bool pass_a(const Tables& tab, const float* span, const Ctl& S, float4* Y, int d,
-                                       int m2, int warp, int grp) {
-  const int sh = S.tma >> 2;
-  const float* sa = span + BLK * slot_block(S, d) + 2 * m2 + sh;
-  const float* sb = span + BLK * slot_block(S, d + DUOS) + 2 * m2 + sh;
+// Pass A for one thread (frames 2d and 2d + 1, role m2): windowed loads,
+// 20-point DFT over m1, twiddle; then, once the previous tile has released
+// the pass buffer (warp 0 waits for its row copies; group barrier), the
+// stores of the 20 outputs.  Returns the group's copy verdict (false: stop).
+// Offline tiles hold one utterance, so frame 2d + 1 starts one hop block
+// after frame 2d (slots of frames past the tile's end hold values whose
+// results are dropped); streaming tiles may pair frames of two streams, so
+// each frame's slots are looked up on their own.
+template <bool kOdd, bool kStream>
+__device__ __forceinline__ bool pass_a(const Tables& tab, const float* span, int eo, const Ctl& S, float4* Y,
+                                       int d, int m2, int warp, int grp) {
+  const int off = 2 * m2 + (S.tma >> 2);
+  const float* pa[3];
+  const float* pb[3];
+  if constexpr (kStream) {
+    const int ba = slot_block(S, 2 * d), bb = slot_block(S, 2 * d + 1);
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      pa[j] = blk_addr(span, eo, ba + j) + off;
+      pb[j] = blk_addr(span, eo, bb + j) + off;
+    }
+  } else {
+    const float* e = span + d * BLK + off;        // hop blocks 2d, 2d + 2
+    const float* o = span + eo + d * BLK + off;   // hop blocks 2d + 1, 2d + 3
+    pa[0] = e;
+    pa[1] = o;
+    pa[2] = e + BLK;
+    pb[0] = o;
+    pb[1] = e + BLK;
+    pb[2] = o + BLK;
+  }
   cx z[N1];
-  window_load<kOdd>(z, sa, sb, tab, m2);
+  window_load<kOdd>(z, pa, pb, tab, m2);
   dft20(z);
 #pragma unroll
   for (int k1 = 1; k1 < N1; ++k1) {
@@ -826,22 +904,23 @@ __device__ __forceinline__ bool pass_a(const Tables& tab, const float* span, con
   }
   return true;
 }
-__device__ __noinline__ bool pass_a_odd(const Tables& tab, const float* span, const Ctl& S, float4* Y, int d,
-                                        int m2, int warp, int grp) {
-  return pass_a<true>(tab, span, S, Y, d, m2, warp, grp);
+__device__ __noinline__ bool pass_a_odd(const Tables& tab, const float* span, int eo, const Ctl& S, float4* Y,
+                                        int d, int m2, int warp, int grp) {
+  return pass_a<true, false>(tab, span, eo, S, Y, d, m2, warp, grp);
 }
 
 // kOddSpans: offline batches in which some utterance starts at an odd float
 // offset from a 16-byte boundary; such spans are read by an out-of-line copy
-// of pass A (elsewhere they fall back to cp.async staging).
-template <bool kDefaultMel, bool kOddSpans>
+// of pass A (elsewhere they fall back to cp.async staging).  kStream: a
+// streaming push (else an offline ragged batch).
+template <bool kDefaultMel, bool kOddSpans, bool kStream>
 __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fused_kernel(const __grid_constant__ Args a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   const int G = blockDim.x / GROUP_THREADS;
   const int grp = threadIdx.x / GROUP_THREADS;
   const int tid = threadIdx.x - grp * GROUP_THREADS;
   const int warp = tid >> 5, lane = tid & 31;
-  // lane -> frame pair d (slots d and d + 16) and role: a half-warp holds 8
+  // lane -> frame pair d (slots 2d and 2d + 1) and role: a half-warp holds 8
   // pairs x 2 adjacent roles, so its strided span reads hit distinct banks
   const int d = ((lane >> 4) << 3) | (lane & 7);
   const int role = 2 * warp + ((lane >> 3) & 1);   // pass A: m2; pass B: k1 pair index
@@ -866,22 +945,33 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
     // with the batch's index map in the parameters, the first tile's span
     // copy (one tensor copy) can leave before the tables are staged
     ctl0->early = 0;
-    if (tile < a.num_tiles && a.mode == 0 && a.meta_inline) {
+    if (!kStream && tile < a.num_tiles && a.meta_inline) {
       setup_offline(*ctl0, a, inline_desc(a, tile), span, kOddSpans);
       if ((ctl0->tma & 3) == 2) {
         ctl0->bar_parity = (armed0++) & 1;
         ctl0->copy_ok = 1;
         ctl0->early = 1;
-        stage_tile(*ctl0, span, tid, a);
+        stage_tile<kStream>(*ctl0, span, tid, a);
       }
     }
+    if (kStream && tile < a.num_tiles) {   // a push: its first tile's groups
+      setup_stream(*ctl0, a, tile);
+      ctl0->copy_ok = 1;
+      ctl0->early = 1;
+    }
+  }
+  if constexpr (kStream) {
+    // a push is one or two tiles per group: its first span copy (cp.async
+    // by the whole group) leaves before the tables are staged
+    group_sync(grp);
+    if (tile < a.num_tiles) stage_tile<kStream>(*ctl0, span, tid, a);
   }
   {  // FFT tables -> shared memory, once per CTA
     const float4* src = reinterpret_cast<const float4*>(a.tables);
     float4* dst = reinterpret_cast<float4*>(smem_raw);
     for (int i = threadIdx.x; i < (int)(sizeof(Tables) / 16); i += blockDim.x) dst[i] = src[i];
   }
-  if (a.mode == 0 && !a.meta_inline) {  // offline: this CTA's tile descriptors, searched in parallel
+  if (!kStream && !a.meta_inline) {  // offline: this CTA's tile descriptors, searched in parallel
     const int rounds = (a.num_tiles + stride - 1) / stride;
     for (int j = threadIdx.x; j < rounds * G; j += blockDim.x) {
       const int t = blockIdx.x * G + (j % G) + (j / G) * stride;
@@ -893,15 +983,15 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
   if (tile < a.num_tiles) {
     if (!ctl0->early) {
       if (tid == COPY_TID) {
-        if (a.mode == 0) setup_offline(*ctl0, a, tile_desc(a, tile), span, kOddSpans);
+        if constexpr (!kStream) setup_offline(*ctl0, a, tile_desc(a, tile), span, kOddSpans);
         else setup_stream(*ctl0, a, tile);
         if (ctl0->tma) ctl0->bar_parity = (armed0++) & 1;
         ctl0->copy_ok = 1;
       }
       group_sync(grp);
-      stage_tile(*ctl0, span, tid, a);
+      stage_tile<kStream>(*ctl0, span, tid, a);
     }
-    if (tid == COPY_TID && a.mode == 0 && tile + stride < a.num_tiles) ctl0->pending = tile_desc(a, tile + stride);
+    if (!kStream && tid == COPY_TID && tile + stride < a.num_tiles) ctl0->pending = tile_desc(a, tile + stride);
   }
   int cur = 0;
   for (; tile < a.num_tiles; tile += stride, cur ^= 1) {
@@ -909,14 +999,15 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
     Ctl& N = cur ? *ctl0 : *ctl1;
     const int next = tile + stride;
     TileDesc nd;   // the next tile's descriptor (used after pass A)
-    if (tid == COPY_TID && a.mode == 0 && next < a.num_tiles) nd = ctl0->pending;
+    if (!kStream && tid == COPY_TID && next < a.num_tiles) nd = ctl0->pending;
     // This tile's span: bulk copies complete on the mbarrier, which every
     // thread polls (bounded: ~65 ms) before it reads the span; a thread that
     // gives up clears the verdict, which the whole group reads after the
     // barrier in pass A.  Per-thread cp.async copies need a barrier to be
     // seen by the other threads.
+    const int polls = a.wait_polls > 0 ? a.wait_polls : (1 << 16);
     if (S.tma) {
-      if (!mbar_wait(&S.bar, S.bar_parity, 1 << 16)) S.copy_ok = 0;
+      if (!mbar_wait(&S.bar, S.bar_parity, polls)) S.copy_ok = 0;
     } else {
       asm volatile("cp.async.wait_all;\n" ::: "memory");
       group_sync(grp);
@@ -924,14 +1015,13 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
     const int ng = S.ngroups;
 
     // ---- streaming: write each owned stream's new carry from the span -----
-    for (int gi = 0; a.mode == 1 && gi < ng; ++gi) {
+    for (int gi = 0; kStream && gi < ng; ++gi) {
       const Group& g = S.groups[gi];
       if (g.carry_len_dst == nullptr) continue;
-      const float* src = span + g.block0 * BLK;
       for (int i = tid; i < g.new_carry_len; i += THREADS) {
         const int p = g.carry_from + i;   // past the staged frames: from the chunk
         const int b = p / HOP;
-        g.carry_dst[i] = p < g.nstage ? src[b * BLK + (p - b * HOP)]
+        g.carry_dst[i] = p < g.nstage ? blk_addr(span, a.eo_off, g.block0 + b)[p - b * HOP]
                                       : g.src1[g.start + p - g.len0];
       }
       if (tid == 0) *g.carry_len_dst = g.new_carry_len;
@@ -944,17 +1034,23 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
       const int sh = S.tma >> 2;   // the slots hold their samples from position sh
       bool ok;
       if constexpr (kOddSpans)
-        ok = (sh & 1) ? pass_a_odd(tab, span, S, Y, d, role, warp, grp)
-                      : pass_a<false>(tab, span, S, Y, d, role, warp, grp);
+        ok = (sh & 1) ? pass_a_odd(tab, span, a.eo_off, S, Y, d, role, warp, grp)
+                      : pass_a<false, kStream>(tab, span, a.eo_off, S, Y, d, role, warp, grp);
       else
-        ok = pass_a<false>(tab, span, S, Y, d, role, warp, grp);
-      if (!ok) {   // a bulk copy never completed: flag it and stop this group
-        if (tid == COPY_TID) atomicExch(a.status, STATUS_COPY_TIMEOUT);
+        ok = pass_a<false, kStream>(tab, span, a.eo_off, S, Y, d, role, warp, grp);
+      if (!ok) {
+        // a span copy did not complete in time: flag it, give copies still
+        // in flight one more bounded wait (a slow copy must land before the
+        // CTA's shared memory is released), and stop this group
+        if (tid == COPY_TID) {
+          atomicExch(a.status, STATUS_COPY_TIMEOUT);
+          mbar_wait(&S.bar, S.bar_parity, polls);
+        }
         break;
       }
     }
     if (tid == COPY_TID && next < a.num_tiles) {   // the next tile's groups
-      if (a.mode == 0) setup_offline(N, a, nd, span, kOddSpans);
+      if constexpr (!kStream) setup_offline(N, a, nd, span, kOddSpans);
       else setup_stream(N, a, next);
       if (N.tma) N.bar_parity = cur ? (armed0++) & 1 : (armed1++) & 1;
       N.copy_ok = 1;
@@ -963,7 +1059,7 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
 
     // every thread has finished reading the span (its values were consumed
     // before the barrier above): fetch the next tile's span meanwhile
-    if (next < a.num_tiles) stage_tile(N, span, tid, a);
+    if (next < a.num_tiles) stage_tile<kStream>(N, span, tid, a);
 
     // ---- pass B: 10-point DFTs over m2, real split, power -----------------
     {
@@ -983,9 +1079,9 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
       dft10(zb);
       group_sync(grp);   // every thread holds its rows: power rows may overwrite Y
       // za[pos10(k2)] = Z[ka + 20 k2], zb[pos10(k2)] = Z[kb + 20 k2].
-      // bin k of slots d and d + 16 at PP[k * TILE] (both bins k and 200 - k
+      // bin k of slots 2d and 2d + 1 at PP[k * TILE] (both bins k and 200 - k
       // of a role have the role's parity)
-      float* PP = Pbuf - TILE + pcol(d, r & 1);
+      float* PP = Pbuf - TILE + pcol(2 * d, r & 1);
       if (warp != 0) {
         // roles 2..9: slot j couples Z[k], k = r + 20 j, with Z[200 - k] = zb[9 - j]
 #pragma unroll
@@ -1060,7 +1156,7 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
         // outside the output tensor and are not written), else one bulk copy
         // per row, issued by the lanes of warp 0
         if (warp == 0) {
-          if (a.mode == 0 && ns == TILE && a.otmap_rows > 0) {
+          if (!kStream && ns == TILE && a.otmap_rows > 0) {
             if (lane == 0) tensor_store_2d(&a.otmap, 0, (int)S.groups[0].out_row, orows);
           } else if (lane < ns) {
             bulk_store(a.out + slot_row(S, lane) * a.n_mels, orows + lane * opitch, (unsigned)a.n_mels * 4u);
@@ -1077,7 +1173,7 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
     }
     // the descriptor of this group's tile after next, found while warp 0
     // issues the row copies (used after the next tile's pass A)
-    if (tid == COPY_TID && a.mode == 0 && next + stride < a.num_tiles) ctl0->pending = tile_desc(a, next + stride);
+    if (!kStream && tid == COPY_TID && next + stride < a.num_tiles) ctl0->pending = tile_desc(a, next + stride);
   }
   if (warp == 0) asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");   // rows written before exit
 }

@@ -119,3 +119,15 @@ def test_noalloc_total_frames_is_the_frame_count(cdll):
     assert f(bad.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), 2) == -1
     assert f(None, 1) == -1
     assert f(p64, -1) == -1
+
+
+def test_fp32_probe_library_exports_its_entry_point():
+    """The FP32 FMA probe bench.py measures the FP32 roof with is built beside
+    the library and exports the call its header declares."""
+    import __graft_entry__
+    path = __graft_entry__._builder().build_peak_probe()
+    lib = ctypes.CDLL(path)
+    src = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", "fp32_peak.h")).read(), flags=re.S)
+    names = set(re.findall(r"\b(fp32_[a-z_]+)\s*\(", src))
+    assert names == {"fp32_fma_probe"}
+    assert hasattr(lib, "fp32_fma_probe")

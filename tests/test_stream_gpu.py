@@ -178,11 +178,14 @@ def test_streaming_full_size_1024x600(plan, lib):
     assert f == F == 4798
     ref = _offline(plan, x)
     assert torch.equal(_bits(got), _bits(ref))
+    # every row of 16 streams against the oracle (76,768 frames), on top of
+    # the bitwise equality with offline for all 1024 streams
     rng = np.random.default_rng(5)
-    for s in rng.choice(S, 4, replace=False):
-        rows = np.sort(rng.choice(F, 200, replace=False))
-        L_, M_ = O.log_mel_frames(xh[s], [0, N], rows)
-        check_against_oracle(got[s].cpu().numpy()[rows], L_, M_)
+    picked = rng.choice(S, 16, replace=False)
+    g = got[torch.from_numpy(picked).cuda()].cpu().numpy()
+    for i, s in enumerate(picked):
+        L_, M_ = O.log_mel(xh[s], return_energy=True)
+        check_against_oracle(g[i], L_, M_)
     assert plan.device_status() == 0
 
 
@@ -208,7 +211,53 @@ def test_long_form_streamed_equals_offline_whole_recording(plan, lib):
     assert got.shape == (O.num_frames(N), 128) == (521_998, 128)
     ref = plan.compute(x, [0, N])
     assert torch.equal(_bits(got), _bits(ref))
-    rows = np.sort(rng.choice(got.shape[0], 400, replace=False))
-    L_, M_ = O.log_mel_frames(pcm, [0, N], rows)
-    check_against_oracle(got.cpu().numpy()[rows], L_, M_)
+    # every row against the oracle, 20,000 rows at a time
+    g = got.cpu().numpy()
+    for r0 in range(0, g.shape[0], 20_000):
+        rows = np.arange(r0, min(g.shape[0], r0 + 20_000))
+        L_, M_ = O.log_mel_frames(pcm, [0, N], rows)
+        check_against_oracle(g[rows], L_, M_)
+    assert plan.device_status() == 0
+
+
+def test_ragged_batch_pushes_equal_offline(plan, lib):
+    """One launch per call, every stream advancing by its own length (0 to
+    5000 samples, mixed across streams and calls): each stream's frames equal
+    the offline log-mel of its concatenated audio bit for bit, and the
+    per-push counts follow the oracle's emission rule."""
+    S, calls = 12, 50
+    sizes = np.array([0, 1, 159, 160, 399, 1280, 1920, 2560, 5000])
+    rng = np.random.default_rng(61)
+    lens = rng.choice(sizes, size=(calls, S))
+    lens[7] = 0                                               # a call where nothing arrives
+    lens[8] = 5000                                            # a call where every stream emits > 28 frames
+    total = lens.sum(0)
+    x = torch.from_numpy(W.stream_signals(S, int(total.max()), seed0=9700)).cuda()
+    st = lib.Stream(plan, S)
+    outs = [[] for _ in range(S)]
+    pos = np.zeros(S, np.int64)
+    for c in range(calls):
+        off = np.concatenate([[0], np.cumsum(lens[c])]).astype(np.int64)
+        packed = torch.cat([x[s, pos[s]:pos[s] + lens[c, s]] for s in range(S)]).contiguous()
+        if packed.numel() == 0:
+            packed = torch.zeros(1, device="cuda")
+        o, n = st.push_batch_ragged(packed, off)
+        for s in range(S):
+            outs[s].append(o[s, :n[s]].clone())
+        pos += lens[c]
+    for s in range(S):
+        counts, carry = O.stream_emit_counts(lens[:, s].tolist())
+        assert [t.shape[0] for t in outs[s]] == counts, s
+        got = torch.cat(outs[s], 0)
+        ref = plan.compute(x[s, :pos[s]].contiguous(), [0, int(pos[s])])
+        assert torch.equal(_bits(got), _bits(ref)), s
+    # the ragged form equals the uniform one when all lengths are equal
+    a, b = lib.Stream(plan, S), lib.Stream(plan, S)
+    L = 1280
+    for i in range(6):
+        chunk = x[:, i * L:(i + 1) * L].contiguous()
+        oa, na = a.push_batch(chunk)
+        ob, nb = b.push_batch_ragged(chunk.reshape(-1), np.arange(S + 1, dtype=np.int64) * L)
+        assert np.array_equal(na, nb)
+        assert torch.equal(_bits(oa[:, :na[0]]), _bits(ob[:, :nb[0]]))
     assert plan.device_status() == 0

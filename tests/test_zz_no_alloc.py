@@ -5,9 +5,14 @@ belongs to another allocator (a serving runtime or host application that
 reserves the GPU's memory and hands out buffers) and real-time audio code
 that must not block in cudaMalloc / cudaFree.  It keeps its tables, ragged
 metadata and tile descriptors in one fixed device array shared by every
-call, so these tests check that two calls in a row -- the first at the
-array's maximum size, the second a small ragged batch that reuses what the
-first left behind -- each match the plan-based logmel_compute.
+call, so these tests check that calls in a row -- the first at the array's
+maximum size (4096 utterances: its index map and tile descriptors fill the
+scratch), then a small ragged batch whose index map travels in the launch,
+then 300 ragged utterances at unaligned offsets that go through the scratch
+again with fewer tiles than the first call left there -- each match the
+plan-based logmel_compute bit for bit, and that a call made after the
+one-time set-up changes neither the device's free memory nor the PyTorch
+allocator's counters.
 
 This file is collected last on purpose: the first call on a device does the
 entry point's one-time set-up, and the tests must pass both alone in a fresh
@@ -23,8 +28,12 @@ from _tolerance import TOL
 MAX_UTT, MAX_TILES = 4096, 32768
 
 
-def _frames(n):
-    return np.where(n >= 400, (n - 400) // 160 + 1, 0)
+def _total_rows(lib, off):
+    offs = np.ascontiguousarray(off, dtype=np.int64)
+    n = lib._lib.logmel_noalloc_total_frames(offs.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+                                             offs.shape[0] - 1)
+    assert n >= 0
+    return int(n)
 
 
 def _noalloc(lib, pcm, off, out, status):
@@ -60,8 +69,21 @@ def _small_ragged_batch(dev):
     return pcm, off
 
 
+def _ragged_beyond_inline(dev):
+    """300 utterances (more than the 256 whose index map fits in the launch)
+    of 401..20000 samples at odd offsets: the index map and the tile
+    descriptors go through the scratch again, with far fewer tiles than the
+    maximum-size call left there."""
+    import torch
+    lens = np.random.default_rng(13).integers(401, 20000, 300).astype(np.int64)
+    off = 1 + np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    g = torch.Generator(device=dev).manual_seed(14)
+    pcm = 0.4 * torch.randn(int(off[-1]) + 3, generator=g, device=dev)
+    return pcm, off
+
+
 @pytest.mark.gpu
-def test_noalloc_matches_compute_on_two_calls_in_a_row():
+def test_noalloc_matches_compute_on_calls_in_a_row():
     import torch
     import log_mel_spectrogram_logmel_b200 as lm
 
@@ -69,9 +91,9 @@ def test_noalloc_matches_compute_on_two_calls_in_a_row():
     torch.cuda.set_device(dev)
     plan = lm.Plan(device=dev)
     status = torch.full((1,), -1, dtype=torch.int32, device=dev)
-    for make in (_max_size_batch, _small_ragged_batch):
+    for make in (_max_size_batch, _small_ragged_batch, _ragged_beyond_inline):
         pcm, off = make(dev)
-        total = int(_frames(np.diff(off)).sum())
+        total = _total_rows(lm, off)
         got = torch.full((total, 128), float("nan"), device=dev)
         assert _noalloc(lm, pcm, off, got, status) == 0
         torch.cuda.synchronize()
@@ -85,6 +107,35 @@ def test_noalloc_matches_compute_on_two_calls_in_a_row():
         assert torch.equal(got.view(torch.int32), want.view(torch.int32)), make.__name__
         del pcm, got, want
     assert plan.device_status() == 0
+
+
+@pytest.mark.gpu
+def test_noalloc_call_allocates_nothing():
+    """After the one-time set-up on the device, a call at the maximum size
+    leaves the device's free memory (cudaMemGetInfo) and the PyTorch caching
+    allocator's counters exactly as they were."""
+    import torch
+    import log_mel_spectrogram_logmel_b200 as lm
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    status = torch.zeros((1,), dtype=torch.int32, device=dev)
+    pcm, off = _max_size_batch(dev)
+    out = torch.empty((_total_rows(lm, off), 128), device=dev)
+    assert _noalloc(lm, pcm, off, out, status) == 0            # set-up (first call on this device)
+    torch.cuda.synchronize()
+    keys = ("allocation.all.allocated", "segment.all.allocated", "reserved_bytes.all.current",
+            "allocated_bytes.all.current")
+    before_stats = {k: torch.cuda.memory_stats(dev).get(k) for k in keys}
+    free_before, _ = torch.cuda.mem_get_info(dev)
+    for _ in range(2):
+        assert _noalloc(lm, pcm, off, out, status) == 0
+    torch.cuda.synchronize()
+    free_after, _ = torch.cuda.mem_get_info(dev)
+    after_stats = {k: torch.cuda.memory_stats(dev).get(k) for k in keys}
+    assert free_after == free_before, (free_before, free_after)
+    assert after_stats == before_stats
+    assert int(status.item()) == 0
 
 
 @pytest.mark.gpu
