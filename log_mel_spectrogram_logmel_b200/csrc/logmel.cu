@@ -189,6 +189,7 @@ struct logmel_plan {
   int device = 0;
   LaunchCfg off{}, str{};    // offline and streaming launch shapes
   Tables* d_tables = nullptr;
+  double* d_fix = nullptr;        // float64 window [400] and (cos, sin) [400] of the accuracy guard
   int* d_status = nullptr;
   unsigned char* d_meta = nullptr;
   size_t meta_cap = 0;
@@ -300,6 +301,14 @@ const char* logmel_status_string(logmel_status s) {
              "(at most 4096 utterances and 32768 tiles of 32 frames)";
   }
   return "unknown status";
+}
+
+// Float64 tables of the accuracy guard's recomputation: the window w[n]
+// (n < 400), then (cos, sin)(2 pi j / 400) (j < 400).
+constexpr int FIX_DOUBLES = NFFT + 2 * NFFT;
+static void build_fix_tables(double* t) {
+  for (int n = 0; n < NFFT; ++n) t[n] = 0.54 - 0.46 * std::cos(2.0 * M_PI * n / (NFFT - 1));
+  for (int j = 0; j < NFFT; ++j) cos_sin_2pi(j, NFFT, &t[NFFT + 2 * j], &t[NFFT + 2 * j + 1]);
 }
 
 static logmel_status build_tables(Tables* t) {
@@ -435,6 +444,8 @@ static cudaError_t launch(const logmel_plan* p, Args& a, int64_t tiles, cudaStre
     }
   }
   a.tables = p->d_tables;
+  a.fix_win = p->d_fix;
+  a.fix_cs = reinterpret_cast<const double2*>(p->d_fix + NFFT);
   a.wait_polls = p->wait_polls;
   a.tx_extra = p->tx_extra;
   a.span_blocks = c.span_blocks;
@@ -515,9 +526,16 @@ logmel_status logmel_plan_create(int sr, int n_fft, int hop, int n_mels, float f
   st = p->default_mel ? setup_kernel<true>(p, sms) : setup_kernel<false>(p, sms);
   if (st != LOGMEL_OK) return fail(st);
   if (cudaMalloc(&p->d_tables, sizeof(Tables)) != cudaSuccess) return fail(LOGMEL_ERR_OOM);
+  if (cudaMalloc(&p->d_fix, sizeof(double) * FIX_DOUBLES) != cudaSuccess) return fail(LOGMEL_ERR_OOM);
   if (cudaMalloc(&p->d_status, sizeof(int)) != cudaSuccess) return fail(LOGMEL_ERR_OOM);
   if (cudaMemcpy(p->d_tables, t, sizeof(Tables), cudaMemcpyHostToDevice) != cudaSuccess)
     return fail(LOGMEL_ERR_CUDA);
+  {
+    std::vector<double> fix(FIX_DOUBLES);
+    build_fix_tables(fix.data());
+    if (cudaMemcpy(p->d_fix, fix.data(), sizeof(double) * FIX_DOUBLES, cudaMemcpyHostToDevice) != cudaSuccess)
+      return fail(LOGMEL_ERR_CUDA);
+  }
   if (cudaMemset(p->d_status, 0, sizeof(int)) != cudaSuccess) return fail(LOGMEL_ERR_CUDA);
   for (int i = 0; i < RING; ++i)
     if (cudaEventCreateWithFlags(&p->ring[i].done, cudaEventDisableTiming) != cudaSuccess)
@@ -534,6 +552,7 @@ void logmel_plan_destroy(logmel_plan* p) {
   cudaSetDevice(p->device);
   cudaDeviceSynchronize();
   cudaFree(p->d_tables);
+  cudaFree(p->d_fix);
   cudaFree(p->d_status);
   cudaFree(p->d_meta);
   cudaFree(p->d_tiles);
@@ -1016,9 +1035,11 @@ constexpr int64_t NOALLOC_MAX_UTT = 4096;     // utterances per call
 constexpr int64_t NOALLOC_MAX_TILES = 32768;  // 32-frame tiles per call (1,048,576 frames)
 constexpr int NOALLOC_MAX_DEVICES = 64;
 
-// Scratch layout: FFT tables | status word | ragged metadata | tile descriptors.
+// Scratch layout: FFT tables | float64 guard tables | status word | ragged
+// metadata | tile descriptors.
 constexpr size_t NA_TABLES_OFF = 0;
-constexpr size_t NA_STATUS_OFF = (sizeof(Tables) + 255) / 256 * 256;
+constexpr size_t NA_FIX_OFF = (sizeof(Tables) + 255) / 256 * 256;
+constexpr size_t NA_STATUS_OFF = NA_FIX_OFF + (sizeof(double) * FIX_DOUBLES + 255) / 256 * 256;
 constexpr size_t NA_META_OFF = NA_STATUS_OFF + 256;
 constexpr size_t NA_META_CAP =   // meta_bytes(NOALLOC_MAX_UTT), rounded up to 256
     (16 * (NOALLOC_MAX_UTT + 1) + ((4 * (NOALLOC_MAX_UTT + 1) + 15) & ~15) + 255) / 256 * 256;
@@ -1076,7 +1097,13 @@ static logmel_status noalloc_setup(int dev, NoAllocDevice& d) {
   if (st != LOGMEL_OK) return st;
   unsigned char* base = static_cast<unsigned char*>(sym);
   CK(cudaMemcpy(base + NA_TABLES_OFF, &t, sizeof(Tables), cudaMemcpyHostToDevice));
+  {
+    double fix[FIX_DOUBLES];
+    build_fix_tables(fix);
+    CK(cudaMemcpy(base + NA_FIX_OFF, fix, sizeof fix, cudaMemcpyHostToDevice));
+  }
   p.d_tables = reinterpret_cast<Tables*>(base + NA_TABLES_OFF);
+  p.d_fix = reinterpret_cast<double*>(base + NA_FIX_OFF);
   p.d_status = reinterpret_cast<int*>(base + NA_STATUS_OFF);
   d.scratch = base;
   d.ready = true;

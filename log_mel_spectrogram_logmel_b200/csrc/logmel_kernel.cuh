@@ -74,6 +74,20 @@ constexpr int INLINE_UTT = 256;           // offline batches up to this size car
 // step 5's floor at mel energy 1e-10); zero energy gives exactly this value.
 constexpr float LOG_FLOOR = -23.025850929940457f;
 
+// Accuracy guard.  fp32 rounding in the FFT leaves every bin with an error
+// of roughly 1e-7 times the frame's RMS bin amplitude (the bins that alias
+// onto it through the 20 x 10 decomposition dominate), so a band whose energy
+// M lies far below the frame's spectral energy S = sum_k |2 X_k|^2 (one-sided,
+// bins 0..200) can miss the 2e-3 log tolerance: e.g. a spectral null 84 dB
+// below the frame's energy.  A frame with a band under RISK_REL * S has its
+// low bands recomputed in float64 by a direct DFT of the frame (mel_fixup).
+// S = 800 E_w, E_w the windowed frame energy, so RISK_REL = 3.75e-10 flags
+// M / E_w < 3e-7.  Measured over every cell of the benchmark workloads, the
+// fp32 error stays within 2 x 3 x 2^-24 / sqrt(M / E_w) in log units, i.e.
+// under 7e-4 above this ratio; errors past 1e-3 occur only below 1e-7.
+constexpr float RISK_REL = 3.75e-10f;
+constexpr float LG2_RISK_REL = -31.312390353265105f;   // log2(RISK_REL)
+
 // FFT tables, built in float64 on the host by the plan and rounded to fp32;
 // one copy in shared memory serves every tile group of a CTA.
 struct __align__(16) Tables {
@@ -130,6 +144,8 @@ struct Args {
   int otmap_rows;       // rows of the output tensor (0: no tensor map)
   int eo_off;           // floats from the even-block region to the odd-block region
   const Tables* tables;
+  const double* fix_win;       // float64 window w[n], n < 400 (accuracy guard)
+  const double2* fix_cs;       // float64 (cos, sin)(2 pi j / 400), j < 400
   TileDesc* tiles;      // offline: per-tile descriptors (written by the kernel's prologue)
   float* out;
   int* status;
@@ -356,9 +372,13 @@ __host__ __device__ constexpr int orow_floats(int n_mels) {
 // Every region starts on a 128-byte boundary: a tensor bulk copy's shared
 // memory address must be 128-byte aligned (the output rows follow the power
 // rows, whose size is a multiple of 128 bytes).
+// After the staged output rows: the frames' spectral energy, one partial sum
+// per pass-B warp and frame slot ([MEL_WARPS][32]; in the pass buffer's free
+// tail for the default 128 bands).
+constexpr int SBUF_FLOATS = MEL_WARPS * TILE;
 __host__ __device__ constexpr int ybuf_bytes_for(int n_mels) {
-  return (((PROWS_FLOATS + TILE * orow_floats(n_mels)) * 4 > YBUF_BYTES
-               ? (PROWS_FLOATS + TILE * orow_floats(n_mels)) * 4
+  return (((PROWS_FLOATS + TILE * orow_floats(n_mels) + SBUF_FLOATS) * 4 > YBUF_BYTES
+               ? (PROWS_FLOATS + TILE * orow_floats(n_mels) + SBUF_FLOATS) * 4
                : YBUF_BYTES) +
           127) / 128 * 128;
 }
@@ -738,11 +758,16 @@ __device__ __forceinline__ void stage_tile(Ctl& S, float* span, int tid, const A
 // ln(max(M, 1e-10)): the hardware base-2 logarithm times ln 2, clamped below
 // at the fp32 value of ln(1e-10) (M >= 1e-10 is normal, so flushing subnormal
 // inputs to zero changes nothing).
-__device__ __forceinline__ float log_floor(float acc) {
-  float l2, r;
-  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(l2) : "f"(acc));
-  // max(ln M, ln 1e-10) = ln max(M, 1e-10); M = 0 gives -inf, hence the
-  // exact floor; a NaN energy stays NaN
+__device__ __forceinline__ float lg2_approx(float x) {
+  float l2;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(l2) : "f"(x));
+  return l2;
+}
+// ln of the energy from its base-2 logarithm, clamped below at the floor:
+// max(ln M, ln 1e-10) = ln max(M, 1e-10); M = 0 gives -inf, hence the exact
+// floor; a NaN energy stays NaN
+__device__ __forceinline__ float ln_floor(float l2) {
+  float r;
   asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(l2 * 0.69314718055994531f), "f"(LOG_FLOOR));
   return r;
 }
@@ -763,25 +788,29 @@ struct MelDot {
   }
 };
 
+// lo2 keeps the smallest lg2 energy over the bands that hold bins (for the
+// accuracy guard); empty bands (always zero) are left out.
 template <int KLO, int M, int NP>
-__device__ __forceinline__ float mel_band(const float (&p)[NP]) {
+__device__ __forceinline__ float mel_band(const float (&p)[NP], float& lo2) {
   constexpr int lo = mel_default::LO[M], cnt = mel_default::CNT[M], wo = mel_default::WOFF[M];
-  return log_floor(MelDot<KLO, lo, wo, 0, cnt, NP>::run(p, 0.f));
+  const float l2 = lg2_approx(MelDot<KLO, lo, wo, 0, cnt, NP>::run(p, 0.f));
+  if constexpr (cnt > 0) lo2 = fminf(lo2, l2);
+  return ln_floor(l2);
 }
 
 // bands [M, MEND) four at a time, one 16-byte store per four bands
 template <int KLO, int M, int MEND, int NP>
 struct MelBands {
-  static __device__ __forceinline__ void run(const float (&p)[NP], float* __restrict__ orow) {
+  static __device__ __forceinline__ void run(const float (&p)[NP], float* __restrict__ orow, float& lo2) {
     if constexpr (M < MEND) {
       static_assert(M % 4 == 0 && MEND % 4 == 0, "warp band ranges are multiples of 4");
       float4 v;
-      v.x = mel_band<KLO, M, NP>(p);
-      v.y = mel_band<KLO, M + 1, NP>(p);
-      v.z = mel_band<KLO, M + 2, NP>(p);
-      v.w = mel_band<KLO, M + 3, NP>(p);
+      v.x = mel_band<KLO, M, NP>(p, lo2);
+      v.y = mel_band<KLO, M + 1, NP>(p, lo2);
+      v.z = mel_band<KLO, M + 2, NP>(p, lo2);
+      v.w = mel_band<KLO, M + 3, NP>(p, lo2);
       *reinterpret_cast<float4*>(orow + M) = v;
-      MelBands<KLO, M + 4, MEND, NP>::run(p, orow);
+      MelBands<KLO, M + 4, MEND, NP>::run(p, orow, lo2);
     }
   }
 };
@@ -803,17 +832,17 @@ __host__ __device__ constexpr int mel_bin_hi(int b0, int b1) {
 
 template <int W>
 __device__ __forceinline__ void mel_default_warp(const float* __restrict__ PE, const float* __restrict__ PO,
-                                                 float* __restrict__ orow) {
+                                                 float* __restrict__ orow, float& lo2) {
   constexpr int B0 = mel_default::WARP_BAND[W], B1 = mel_default::WARP_BAND[W + 1];
   constexpr int KLO = mel_bin_lo(B0, B1), KHI = mel_bin_hi(B0, B1), NP = KHI - KLO + 1;
   float p[NP];
 #pragma unroll
   for (int i = 0; i < NP; ++i) p[i] = (((KLO + i) & 1) ? PO : PE)[(KLO + i) * TILE];   // each bin read once
-  MelBands<KLO, B0, B1, NP>::run(p, orow);
+  MelBands<KLO, B0, B1, NP>::run(p, orow, lo2);
 }
 
 __device__ __forceinline__ void mel_generic_warp(const Args& a, int w, const float* PE, const float* PO,
-                                                 float* orow) {
+                                                 float* orow, float& lo2) {
   const int mb = a.warp_band[w], me = a.warp_band[w + 1];
   for (int m = mb; m < me; ++m) {
     const int lo = a.mel_lo[m], cnt = a.mel_cnt[m], wo = a.mel_woff[m];
@@ -822,7 +851,75 @@ __device__ __forceinline__ void mel_generic_warp(const Args& a, int w, const flo
       const int k = lo + j;
       acc = fmaf(a.mel_w[wo + j], ((k & 1) ? PO : PE)[k * TILE], acc);
     }
-    orow[m] = log_floor(acc);
+    const float l2 = lg2_approx(acc);
+    if (cnt > 0) lo2 = fminf(lo2, l2);
+    orow[m] = ln_floor(l2);
+  }
+}
+
+// Float64 recomputation of flagged bands of one warp's band range [b0, b1).
+// For every lane (frame slot) whose smallest band energy fell under its
+// threshold thr (lg2 units), the whole warp recomputes each of its bands
+// still under thr from the frame's samples in global memory, as the
+// pipeline defines them: the window, a direct DFT of each bin of the band
+// (lane t sums samples t, t + 32, ..., a fixed shuffle tree adds the
+// lanes), the band's weighted power sum and ln(max(M, 1e-10)), which
+// replaces the staged value.  The result depends only on the frame's
+// samples, so a frame gives the same bits in every tile and slot.  Rare,
+// and kept out of line so that the common path stays small.
+__device__ __noinline__ void mel_fixup(const Args& a, const Ctl& S, float* orows, int opitch, int b0, int b1,
+                                       float thr, bool risk, int lane) {
+  constexpr unsigned FULL = 0xffffffffu;
+  constexpr int T = (NFFT + 31) / 32;   // samples per lane
+  __syncwarp();                         // every lane's staged row is visible to the warp
+  unsigned todo = __ballot_sync(FULL, risk);
+  while (todo) {
+    const int f = __ffs(todo) - 1;
+    todo &= todo - 1;
+    const float thr_f = __shfl_sync(FULL, thr, f);
+    int gi = 0;   // the group (source) holding frame slot f
+    for (int i = 0; i < S.ngroups; ++i)
+      if (f >= S.groups[i].slot0 && f < S.groups[i].slot0 + S.groups[i].nframes) gi = i;
+    const Group& g = S.groups[gi];
+    const int64_t base = g.start + (int64_t)HOP * (f - g.slot0);
+    double xw[T];
+#pragma unroll
+    for (int t = 0; t < T; ++t) {
+      const int n = lane + 32 * t;
+      xw[t] = n < NFFT ? (double)src_at(g, base + n) * a.fix_win[n] : 0.0;
+    }
+    float* orow = orows + f * opitch;
+#pragma unroll 1
+    for (int m = b0; m < b1; ++m) {
+      const int cnt = a.mel_cnt[m];
+      if (cnt == 0 || !(orow[m] * 1.4426950408889634f < thr_f)) continue;
+      double msum = 0.0;
+#pragma unroll 1
+      for (int j = 0; j < cnt; ++j) {
+        const int k = a.mel_lo[m] + j;
+        double re = 0.0, im = 0.0;
+        int idx = (k * lane) % NFFT;   // (k n) mod 400 for n = lane + 32 t
+        const int step = (k * 32) % NFFT;
+#pragma unroll
+        for (int t = 0; t < T; ++t) {
+          const double2 cs = a.fix_cs[idx];
+          re = fma(xw[t], cs.x, re);
+          im = fma(xw[t], cs.y, im);
+          idx += step;
+          if (idx >= NFFT) idx -= NFFT;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          re += __shfl_xor_sync(FULL, re, o);
+          im += __shfl_xor_sync(FULL, im, o);
+        }
+        // the weights carry the factor 1/4 of |2 X|^2
+        msum = fma(4.0 * (double)a.mel_w[a.mel_woff[m] + j], re * re + im * im, msum);
+      }
+      __syncwarp();
+      if (lane == 0) orow[m] = msum < 1e-10 ? LOG_FLOOR : fmaxf(logf((float)msum), LOG_FLOOR);
+      __syncwarp();
+    }
   }
 }
 
@@ -934,6 +1031,7 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
   float* const span = reinterpret_cast<float*>(gbase + 2 * CTL_BYTES + a.ybuf_bytes);
   float* const Pbuf = reinterpret_cast<float*>(Y);   // power rows, after pass B has read Y
   float* const orows = Pbuf + PROWS_FLOATS;          // staged output rows, after the power rows
+  float* const Sbuf = orows + TILE * orow_floats(a.n_mels);   // [MEL_WARPS][32]: frames' spectral energy
   const int opitch = orow_floats(a.n_mels);
   int tile = blockIdx.x * G + grp;
   int armed0 = 0, armed1 = 0;   // COPY_TID: bulk-copy uses of each control buffer
@@ -1014,18 +1112,6 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
     }
     const int ng = S.ngroups;
 
-    // ---- streaming: write each owned stream's new carry from the span -----
-    for (int gi = 0; kStream && gi < ng; ++gi) {
-      const Group& g = S.groups[gi];
-      if (g.carry_len_dst == nullptr) continue;
-      for (int i = tid; i < g.new_carry_len; i += THREADS) {
-        const int p = g.carry_from + i;   // past the staged frames: from the chunk
-        const int b = p / HOP;
-        g.carry_dst[i] = p < g.nstage ? blk_addr(span, a.eo_off, g.block0 + b)[p - b * HOP]
-                                      : g.src1[g.start + p - g.len0];
-      }
-      if (tid == 0) *g.carry_len_dst = g.new_carry_len;
-    }
 
     // ---- pass A: window, 20-point DFTs over m1, twiddle --------------------
     // (spans staged at an odd float offset take a separate, out-of-line copy
@@ -1059,7 +1145,8 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
 
     // every thread has finished reading the span (its values were consumed
     // before the barrier above): fetch the next tile's span meanwhile
-    if (next < a.num_tiles) stage_tile<kStream>(N, span, tid, a);
+    // (streaming: after the tile's carries are written, at its end)
+    if (!kStream && next < a.num_tiles) stage_tile<kStream>(N, span, tid, a);
 
     // ---- pass B: 10-point DFTs over m2, real split, power -----------------
     {
@@ -1082,6 +1169,9 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
       // bin k of slots 2d and 2d + 1 at PP[k * TILE] (both bins k and 200 - k
       // of a role have the role's parity)
       float* PP = Pbuf - TILE + pcol(2 * d, r & 1);
+      // q: this thread's share of the frames' one-sided spectral energy
+      // sum_k |2 X_k|^2 (k = 0..200), for the mel stage's accuracy guard
+      float2 q = make_float2(0.f, 0.f);
       if (warp != 0) {
         // roles 2..9: slot j couples Z[k], k = r + 20 j, with Z[200 - k] = zb[9 - j]
 #pragma unroll
@@ -1091,6 +1181,7 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
           split_power(tab, za[pos10(j)], zb[pos10(9 - j)], k, pk, pm);
           *reinterpret_cast<float2*>(PP + k * TILE) = pk;
           *reinterpret_cast<float2*>(PP + (200 - k) * TILE) = pm;
+          q = add2(q, add2(pk, pm));
         }
       } else {
         // roles 0 and 1 share this warp; role 0 owns the self-paired tasks
@@ -1110,14 +1201,21 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
             *reinterpret_cast<float2*>(PP + k * TILE) = pk;
             *reinterpret_cast<float2*>(PP + (200 - k) * TILE) = pm;
           }
+          q = add2(q, add2(pk, pm));   // k = 0: bins 0 and 200
         }
         if (r0) {
           const cx z = za[pos10(5)];
           const float2 tr = add2(z.re, z.re), ti = add2(z.im, z.im);
           const float2 p = fma2(ti, ti, mul2(tr, tr));
           *reinterpret_cast<float2*>(PP + 100 * TILE) = p;
+          q = add2(q, p);
         }
       }
+      // the pair's two roles in this warp (lanes l and l ^ 8) add their
+      // shares; one of them leaves the warp's partial sum for the pair
+      q.x += __shfl_xor_sync(0xffffffffu, q.x, 8);
+      q.y += __shfl_xor_sync(0xffffffffu, q.y, 8);
+      if (((lane >> 3) & 1) == 0) *reinterpret_cast<float2*>(Sbuf + warp * TILE + 2 * d) = q;
     }
     group_sync(grp);
 
@@ -1126,26 +1224,39 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
       const float* PE = Pbuf - TILE + pcol(lane, 0);
       const float* PO = Pbuf - TILE + pcol(lane, 1);
       float* orow = orows + lane * opitch;
+      float lo2 = __int_as_float(0x7f800000);   // +inf: the smallest lg2 band energy so far
       if constexpr (kDefaultMel) {
         switch (warp) {
-          case 0: mel_default_warp<0>(PE, PO, orow); break;
-          case 1: mel_default_warp<1>(PE, PO, orow); break;
-          case 2: mel_default_warp<2>(PE, PO, orow); break;
-          case 3: mel_default_warp<3>(PE, PO, orow); break;
-          default: mel_default_warp<4>(PE, PO, orow); break;
+          case 0: mel_default_warp<0>(PE, PO, orow, lo2); break;
+          case 1: mel_default_warp<1>(PE, PO, orow, lo2); break;
+          case 2: mel_default_warp<2>(PE, PO, orow, lo2); break;
+          case 3: mel_default_warp<3>(PE, PO, orow, lo2); break;
+          default: mel_default_warp<4>(PE, PO, orow, lo2); break;
         }
       } else {
-        mel_generic_warp(a, warp, PE, PO, orow);
+        mel_generic_warp(a, warp, PE, PO, orow, lo2);
       }
+      // accuracy guard: the frame's spectral energy S (the five pass-B warps'
+      // partial sums) and the threshold lg2(RISK_REL * S); slots past the
+      // tile's frames are never flagged
+      float esum = 0.f;
+#pragma unroll
+      for (int w = 0; w < MEL_WARPS; ++w) esum += Sbuf[w * TILE + lane];
+      const float thr = lane < S.nslots ? lg2_approx(esum) + LG2_RISK_REL : __int_as_float(0xff800000);
+      const bool risk = lo2 < thr;
+      if (__any_sync(0xffffffffu, risk))
+        mel_fixup(a, S, orows, opitch, a.warp_band[warp], a.warp_band[warp + 1], thr, risk, lane);
     }
-    if (a.bulk_store) {
-      // the staged rows precede the bulk copies reading them; only warp 0,
-      // which issues the copies, waits for every warp's rows
-      fence_async_smem();
+    if (a.bulk_store) fence_async_smem();   // the staged rows precede the bulk copies reading them
+    if (a.bulk_store && !kStream) {
+      // only warp 0, which issues the copies, waits for every warp's rows
       if (warp == 0) group_wait2(grp);
       else group_arrive2(grp);
     } else {
-      group_sync(grp);   // every warp stores rows written by every warp
+      // every warp stores rows written by every warp; streaming: no thread
+      // overwrites a carry (below) while a warp's accuracy guard may still
+      // read the frames' samples from it
+      group_sync(grp);
     }
 
     // ---- store: the staged rows of the tile's frames ---------------------
@@ -1174,6 +1285,26 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
     // the descriptor of this group's tile after next, found while warp 0
     // issues the row copies (used after the next tile's pass A)
     if (!kStream && tid == COPY_TID && next + stride < a.num_tiles) ctl0->pending = tile_desc(a, next + stride);
+    if constexpr (kStream) {
+      // each owned stream's new carry, from the span (the mel stage's
+      // accuracy guard may have read the frames' samples from the old
+      // carry), then the next tile's span
+      for (int gi = 0; gi < ng; ++gi) {
+        const Group& g = S.groups[gi];
+        if (g.carry_len_dst == nullptr) continue;
+        for (int i = tid; i < g.new_carry_len; i += THREADS) {
+          const int p = g.carry_from + i;   // past the staged frames: from the chunk
+          const int b = p / HOP;
+          g.carry_dst[i] = p < g.nstage ? blk_addr(span, a.eo_off, g.block0 + b)[p - b * HOP]
+                                        : g.src1[g.start + p - g.len0];
+        }
+        if (tid == 0) *g.carry_len_dst = g.new_carry_len;
+      }
+      if (next < a.num_tiles) {
+        group_sync(grp);   // the span has been read
+        stage_tile<kStream>(N, span, tid, a);
+      }
+    }
   }
   if (warp == 0) asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");   // rows written before exit
 }
