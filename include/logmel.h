@@ -224,7 +224,7 @@ logmel_status logmel_stream_reset(logmel_stream* st, int stream_id, void* stream
  *
  * Scratch and limits: the FFT tables, the status word, the ragged metadata
  * and the tile descriptors live in one fixed array in device memory (about
- * 600 KB, held by every GPU that loads this library until the process
+ * 740 KB, held by every GPU that loads this library until the process
  * exits).  A call takes at most 4096 utterances and 32768 tiles, where
  * utterance u needs ceil(frames_u / 32) tiles (for example 4096 utterances
  * of up to 2.5 s, 64 of 30 s, or one of up to 2.9 h); beyond either limit it

@@ -190,6 +190,8 @@ struct logmel_plan {
   LaunchCfg off{}, str{};    // offline and streaming launch shapes
   Tables* d_tables = nullptr;
   double* d_fix = nullptr;        // float64 window [400] and (cos, sin) [400] of the accuracy guard
+  FixItem* d_fixq = nullptr;      // deferred accuracy-guard frames, FIXQ_CAP per offline tile group
+  int fixq_groups = 0;            // tile groups d_fixq holds (0: none; recompute inside the tile)
   int* d_status = nullptr;
   unsigned char* d_meta = nullptr;
   size_t meta_cap = 0;
@@ -405,8 +407,8 @@ static void shape_launch(LaunchCfg& c, int span_blocks, int n_mels, int max_smem
   c.ybuf_bytes = ybuf_bytes_for(n_mels);
   c.group_bytes = group_bytes_for(span_blocks, n_mels);
   c.groups = MAX_TILE_GROUPS;
-  while (c.groups > 1 && TAB_BYTES + (size_t)c.groups * c.group_bytes > (size_t)max_smem) --c.groups;
-  c.smem = TAB_BYTES + (size_t)c.groups * c.group_bytes;
+  while (c.groups > 1 && TAB_BYTES + (size_t)c.groups * c.group_bytes + FIXN_BYTES > (size_t)max_smem) --c.groups;
+  c.smem = TAB_BYTES + (size_t)c.groups * c.group_bytes + FIXN_BYTES;
 }
 
 template <bool kDefault>
@@ -460,6 +462,11 @@ static cudaError_t launch(const logmel_plan* p, Args& a, int64_t tiles, cudaStre
   std::memcpy(a.warp_band, p->mel.warp_band, sizeof a.warp_band);
   const int grid = (int)std::min<int64_t>((tiles + c.groups - 1) / c.groups, c.max_ctas);
   const int block = c.groups * GROUP_THREADS;
+  // offline: each tile group queues its flagged frames (when the queue
+  // covers every group of the grid)
+  const bool fixq = a.mode == 0 && p->d_fixq != nullptr && (int64_t)grid * c.groups <= p->fixq_groups;
+  a.fixq = fixq ? p->d_fixq : nullptr;
+  a.fixq_cap = fixq ? FIXQ_CAP : 0;
   if (a.mode == 1) {
     if (p->default_mel) logmel_fused_kernel<true, false, true><<<grid, block, c.smem, s>>>(a);
     else logmel_fused_kernel<false, false, true><<<grid, block, c.smem, s>>>(a);
@@ -528,6 +535,9 @@ logmel_status logmel_plan_create(int sr, int n_fft, int hop, int n_mels, float f
   if (cudaMalloc(&p->d_tables, sizeof(Tables)) != cudaSuccess) return fail(LOGMEL_ERR_OOM);
   if (cudaMalloc(&p->d_fix, sizeof(double) * FIX_DOUBLES) != cudaSuccess) return fail(LOGMEL_ERR_OOM);
   if (cudaMalloc(&p->d_status, sizeof(int)) != cudaSuccess) return fail(LOGMEL_ERR_OOM);
+  p->fixq_groups = p->off.max_ctas * p->off.groups;
+  if (cudaMalloc(&p->d_fixq, sizeof(FixItem) * FIXQ_CAP * (size_t)p->fixq_groups) != cudaSuccess)
+    return fail(LOGMEL_ERR_OOM);
   if (cudaMemcpy(p->d_tables, t, sizeof(Tables), cudaMemcpyHostToDevice) != cudaSuccess)
     return fail(LOGMEL_ERR_CUDA);
   {
@@ -553,6 +563,7 @@ void logmel_plan_destroy(logmel_plan* p) {
   cudaDeviceSynchronize();
   cudaFree(p->d_tables);
   cudaFree(p->d_fix);
+  cudaFree(p->d_fixq);
   cudaFree(p->d_status);
   cudaFree(p->d_meta);
   cudaFree(p->d_tiles);
@@ -644,9 +655,23 @@ logmel_status logmel_compute(logmel_plan* p, const float* pcm, const int64_t* of
   if (tiles >= INT32_MAX || frames >= INT32_MAX) return LOGMEL_ERR_INPUT_TOO_LONG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   Args a{};
+  // the tile descriptors, which the kernel's prologue writes and its tile
+  // loop reads
+  if ((size_t)tiles > p->tiles_cap) {
+    CK(cudaDeviceSynchronize());
+    CK(cudaFree(p->d_tiles));
+    p->d_tiles = nullptr;
+    const size_t cap = std::max<size_t>((size_t)tiles, 1024);
+    if (cudaMalloc(&p->d_tiles, cap * sizeof(TileDesc)) != cudaSuccess) {
+      p->tiles_cap = 0;
+      return LOGMEL_ERR_OOM;
+    }
+    p->tiles_cap = cap;
+  }
+  a.tiles = p->d_tiles;
   if (n_utt <= INLINE_UTT) {
     // small batches: the ragged index map travels in the launch parameters,
-    // and the kernel finds each tile's utterance there (no copy, no scratch)
+    // and the kernel finds each tile's utterance there (no metadata copy)
     a.meta_inline = 1;
     a.im_frame_off[0] = 0;
     a.im_tile_off[0] = 0;
@@ -660,17 +685,6 @@ logmel_status logmel_compute(logmel_plan* p, const float* pcm, const int64_t* of
     const size_t bytes = meta_bytes(n_utt);
     st = ensure_meta(p, bytes);
     if (st != LOGMEL_OK) return st;
-    if ((size_t)tiles > p->tiles_cap) {
-      CK(cudaDeviceSynchronize());
-      CK(cudaFree(p->d_tiles));
-      p->d_tiles = nullptr;
-      const size_t cap = std::max<size_t>((size_t)tiles, 1024);
-      if (cudaMalloc(&p->d_tiles, cap * sizeof(TileDesc)) != cudaSuccess) {
-        p->tiles_cap = 0;
-        return LOGMEL_ERR_OOM;
-      }
-      p->tiles_cap = cap;
-    }
     PinnedSlot& slot = p->ring[p->ring_next];
     p->ring_next = (p->ring_next + 1) % RING;
     if (slot.used) CK(cudaEventSynchronize(slot.done));
@@ -690,7 +704,6 @@ logmel_status logmel_compute(logmel_plan* p, const float* pcm, const int64_t* of
     a.sample_off = dv.sample_off;
     a.frame_off = dv.frame_off;
     a.tile_off = dv.tile_off;
-    a.tiles = p->d_tiles;
   }
   a.out = out;
   a.status = p->d_status;
@@ -1036,7 +1049,7 @@ constexpr int64_t NOALLOC_MAX_TILES = 32768;  // 32-frame tiles per call (1,048,
 constexpr int NOALLOC_MAX_DEVICES = 64;
 
 // Scratch layout: FFT tables | float64 guard tables | status word | ragged
-// metadata | tile descriptors.
+// metadata | tile descriptors | deferred guard frames.
 constexpr size_t NA_TABLES_OFF = 0;
 constexpr size_t NA_FIX_OFF = (sizeof(Tables) + 255) / 256 * 256;
 constexpr size_t NA_STATUS_OFF = NA_FIX_OFF + (sizeof(double) * FIX_DOUBLES + 255) / 256 * 256;
@@ -1044,12 +1057,14 @@ constexpr size_t NA_META_OFF = NA_STATUS_OFF + 256;
 constexpr size_t NA_META_CAP =   // meta_bytes(NOALLOC_MAX_UTT), rounded up to 256
     (16 * (NOALLOC_MAX_UTT + 1) + ((4 * (NOALLOC_MAX_UTT + 1) + 15) & ~15) + 255) / 256 * 256;
 constexpr size_t NA_TILES_OFF = NA_META_OFF + NA_META_CAP;
-constexpr size_t NA_SCRATCH_BYTES = NA_TILES_OFF + NOALLOC_MAX_TILES * sizeof(TileDesc);
-static_assert(NA_SCRATCH_BYTES < 640 * 1024, "no-alloc scratch is meant to stay modest");
+constexpr int NA_FIXQ_GROUPS = 512;   // tile groups with a deferred-frame queue (148 SMs x 3 on a B200)
+constexpr size_t NA_FIXQ_OFF = NA_TILES_OFF + NOALLOC_MAX_TILES * sizeof(TileDesc);
+constexpr size_t NA_SCRATCH_BYTES = NA_FIXQ_OFF + (size_t)NA_FIXQ_GROUPS * FIXQ_CAP * sizeof(FixItem);
+static_assert(NA_SCRATCH_BYTES < 768 * 1024, "no-alloc scratch is meant to stay modest");
 
 }  // namespace
 
-// The fixed device scratch (about 600 KB; every GPU that loads this library
+// The fixed device scratch (about 740 KB; every GPU that loads this library
 // holds one copy until the process exits).  In host code this name is only
 // a stand-in for the symbol: its device address comes from
 // cudaGetSymbolAddress, once per device, in noalloc_setup.
@@ -1105,6 +1120,8 @@ static logmel_status noalloc_setup(int dev, NoAllocDevice& d) {
   p.d_tables = reinterpret_cast<Tables*>(base + NA_TABLES_OFF);
   p.d_fix = reinterpret_cast<double*>(base + NA_FIX_OFF);
   p.d_status = reinterpret_cast<int*>(base + NA_STATUS_OFF);
+  p.d_fixq = reinterpret_cast<FixItem*>(base + NA_FIXQ_OFF);
+  p.fixq_groups = NA_FIXQ_GROUPS;
   d.scratch = base;
   d.ready = true;
   return LOGMEL_OK;
@@ -1158,7 +1175,7 @@ extern "C" logmel_status logmel_compute_noalloc(const float* pcm, const int64_t*
   } else {
     // larger batches: the index map in the static host buffer, copied into
     // the scratch (a copy from pageable memory has consumed its source when
-    // it returns); the kernel writes the tile descriptors into the scratch
+    // it returns)
     const size_t bytes = meta_bytes(n_utt);
     MetaView hv = meta_view(g_noalloc_meta, n_utt);
     hv.frame_off[0] = 0;
@@ -1175,8 +1192,8 @@ extern "C" logmel_status logmel_compute_noalloc(const float* pcm, const int64_t*
     a.sample_off = dv.sample_off;
     a.frame_off = dv.frame_off;
     a.tile_off = dv.tile_off;
-    a.tiles = reinterpret_cast<TileDesc*>(d.scratch + NA_TILES_OFF);
   }
+  a.tiles = reinterpret_cast<TileDesc*>(d.scratch + NA_TILES_OFF);
   // the status word starts at zero on every call; the tile descriptors are
   // rewritten by the kernel before it reads them, so they need no clearing
   int* status = device_status ? device_status : d.plan.d_status;

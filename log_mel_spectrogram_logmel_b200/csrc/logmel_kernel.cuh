@@ -80,7 +80,7 @@ constexpr float LOG_FLOOR = -23.025850929940457f;
 // M lies far below the frame's spectral energy S = sum_k |2 X_k|^2 (one-sided,
 // bins 0..200) can miss the 2e-3 log tolerance: e.g. a spectral null 84 dB
 // below the frame's energy.  A frame with a band under RISK_REL * S has its
-// low bands recomputed in float64 by a direct DFT of the frame (mel_fixup).
+// flagged bands recomputed in float64 by a direct DFT of the frame (fix_frame).
 // S = 800 E_w, E_w the windowed frame energy, so RISK_REL = 3.75e-10 flags
 // M / E_w < 3e-7.  Measured over every cell of the benchmark workloads, the
 // fp32 error stays within 2 x 3 x 2^-24 / sqrt(M / E_w) in log units, i.e.
@@ -121,6 +121,16 @@ struct TileDesc {
   int out_row;        // output row of the tile's first frame
   int nframes;
 };
+
+// A frame whose bands the accuracy guard recomputes after the group's last
+// tile: its first sample in pcm, its output row and its threshold (lg2 units).
+struct __align__(16) FixItem {
+  int64_t src;
+  int row;
+  float thr;
+};
+constexpr int FIXQ_CAP = 16;   // deferred frames per tile group
+constexpr int FIXN_BYTES = 16;  // shared memory after the groups' regions: each group's count of deferred frames
 
 struct Args {
   // offline: tensor views of the PCM for the tile copies, one per parity q
@@ -184,6 +194,11 @@ struct Args {
   // sets them to make the wait run out while every real copy still lands)
   int wait_polls;
   int tx_extra;
+  // offline accuracy guard, deferred: each tile group's frames to recompute
+  // (fixq + gid * fixq_cap, gid = blockIdx.x * groups + group), handled after
+  // its last tile; fixq_cap == 0: recomputed inside their tile
+  FixItem* fixq;
+  int fixq_cap;
   // filterbank (per plan): weights / 4 (the real split yields |2 X|^2), and
   // for the generic (non-default) layout the band structure
   float mel_w[MAX_WEIGHTS];
@@ -351,7 +366,6 @@ struct __align__(16) Ctl {
   int copy_ok;              // verdict on the bulk copies (0: a thread's bounded wait gave up)
   int tmap_row;             // tensor copies: the span's first 160-sample row of the buffer
   int tmap_y;               // and its start class (-1: on a row; see Args::tmap)
-  TileDesc pending;         // offline: the descriptor of the group's tile after next
   int early;                // 1: the first tile's copy was issued before the prologue's barrier
 };
 constexpr int TAB_BYTES = (int)((sizeof(Tables) + 127) / 128 * 128);
@@ -373,9 +387,10 @@ __host__ __device__ constexpr int orow_floats(int n_mels) {
 // memory address must be 128-byte aligned (the output rows follow the power
 // rows, whose size is a multiple of 128 bytes).
 // After the staged output rows: the frames' spectral energy, one partial sum
-// per pass-B warp and frame slot ([MEL_WARPS][32]; in the pass buffer's free
-// tail for the default 128 bands).
-constexpr int SBUF_FLOATS = MEL_WARPS * TILE;
+// per pass-B warp and frame slot ([MEL_WARPS][32]), then the accuracy guard's
+// threshold per frame slot [32] and the tile's mask of flagged slots (in the
+// pass buffer's free tail for the default 128 bands).
+constexpr int SBUF_FLOATS = MEL_WARPS * TILE + TILE + 4;
 __host__ __device__ constexpr int ybuf_bytes_for(int n_mels) {
   return (((PROWS_FLOATS + TILE * orow_floats(n_mels) + SBUF_FLOATS) * 4 > YBUF_BYTES
                ? (PROWS_FLOATS + TILE * orow_floats(n_mels) + SBUF_FLOATS) * 4
@@ -403,7 +418,7 @@ __device__ __forceinline__ const float* blk_addr(const float* span, int eo, int 
 }
 // Three offline tile groups of the default 128-band layout must fit in the
 // 232,448 bytes of shared memory an sm_100 CTA may opt into (15 warps per SM).
-static_assert(TAB_BYTES + MAX_TILE_GROUPS * group_bytes_for(OFFLINE_SPAN_BLOCKS, 128) <= 232448,
+static_assert(TAB_BYTES + MAX_TILE_GROUPS * group_bytes_for(OFFLINE_SPAN_BLOCKS, 128) + FIXN_BYTES <= 232448,
               "three default tile groups per CTA");
 
 // Power-row column of frame slot f for a bin of parity par: the frames 2p
@@ -558,10 +573,11 @@ __device__ __noinline__ TileDesc inline_desc(const Args& a, int tile) {
   t.nframes = min(TILE, a.im_frame_off[u + 1] - a.im_frame_off[u] - f0);
   return t;
 }
-// Descriptor of offline tile t: searched in the parameters, or written by
-// the prologue into the descriptor scratch.
-__device__ __forceinline__ TileDesc tile_desc(const Args& a, int t) {
-  return a.meta_inline ? inline_desc(a, t) : a.tiles[t];
+// Descriptor of offline tile t, searched in the parameters or in the
+// device metadata (the prologue writes each CTA's tiles' descriptors into the
+// descriptor scratch, which the tile loop then reads).
+__device__ __forceinline__ TileDesc search_desc(const Args& a, int t) {
+  return a.meta_inline ? inline_desc(a, t) : offline_desc(a, t);
 }
 
 // odd_ok: the kernel can read spans staged at an odd float offset.
@@ -857,70 +873,78 @@ __device__ __forceinline__ void mel_generic_warp(const Args& a, int w, const flo
   }
 }
 
-// Float64 recomputation of flagged bands of one warp's band range [b0, b1).
-// For every lane (frame slot) whose smallest band energy fell under its
-// threshold thr (lg2 units), the whole warp recomputes each of its bands
-// still under thr from the frame's samples in global memory, as the
-// pipeline defines them: the window, a direct DFT of each bin of the band
-// (lane t sums samples t, t + 32, ..., a fixed shuffle tree adds the
-// lanes), the band's weighted power sum and ln(max(M, 1e-10)), which
-// replaces the staged value.  The result depends only on the frame's
-// samples, so a frame gives the same bits in every tile and slot.  Rare,
-// and kept out of line so that the common path stays small.
-__device__ __noinline__ void mel_fixup(const Args& a, const Ctl& S, float* orows, int opitch, int b0, int b1,
-                                       float thr, bool risk, int lane) {
+// Float64 recomputation of one frame's flagged bands (accuracy guard), by
+// one warp: every band whose value in the frame's row lies under the frame's
+// threshold thr (lg2 units) is recomputed from the frame's samples as the
+// pipeline defines it: the window, a direct DFT of each bin of the band (lane
+// t sums samples t, t + 32, ..., its angle advanced by a float64 rotation of
+// 32 samples; a fixed shuffle tree adds the lanes), the band's weighted power
+// sum and ln(max(M, 1e-10)), which replaces the row's value (a band without
+// bins keeps the floor).  The row is a staged row in shared memory or the
+// output row in global memory.  Sample n of the frame is sample base + n of
+// the concatenation src0[0 .. len0) ++ src1.  Every load is issued before the
+// first use (branch-free addresses), so a cold frame costs one memory latency
+// rather than one per sample.  The result depends only on the frame's
+// samples, so a frame gives the same bits whichever tile, slot, kernel or time
+// recomputes it.  Rare: out of line, with the band and bin loops rolled.
+__device__ __noinline__ void fix_frame(const Args& a, const float* src0, int64_t len0, const float* src1, int64_t base,
+                                       float* row, float thr, int lane) {
   constexpr unsigned FULL = 0xffffffffu;
-  constexpr int T = (NFFT + 31) / 32;   // samples per lane
-  __syncwarp();                         // every lane's staged row is visible to the warp
-  unsigned todo = __ballot_sync(FULL, risk);
-  while (todo) {
-    const int f = __ffs(todo) - 1;
-    todo &= todo - 1;
-    const float thr_f = __shfl_sync(FULL, thr, f);
-    int gi = 0;   // the group (source) holding frame slot f
-    for (int i = 0; i < S.ngroups; ++i)
-      if (f >= S.groups[i].slot0 && f < S.groups[i].slot0 + S.groups[i].nframes) gi = i;
-    const Group& g = S.groups[gi];
-    const int64_t base = g.start + (int64_t)HOP * (f - g.slot0);
-    double xw[T];
+  constexpr int T = (NFFT + 31) / 32;          // samples per lane
+  constexpr int C = (MAX_MELS + 31) / 32;      // band chunks of 32
+  float x[T];
+  double w[T];
 #pragma unroll
-    for (int t = 0; t < T; ++t) {
-      const int n = lane + 32 * t;
-      xw[t] = n < NFFT ? (double)src_at(g, base + n) * a.fix_win[n] : 0.0;
-    }
-    float* orow = orows + f * opitch;
-#pragma unroll 1
-    for (int m = b0; m < b1; ++m) {
-      const int cnt = a.mel_cnt[m];
-      if (cnt == 0 || !(orow[m] * 1.4426950408889634f < thr_f)) continue;
+  for (int t = 0; t < T; ++t) {
+    const int n = min(lane + 32 * t, NFFT - 1);
+    const int64_t pos = base + n;
+    x[t] = *(pos < len0 ? src0 + pos : src1 + (pos - len0));
+    w[t] = a.fix_win[n];
+  }
+  float v[C];
+#pragma unroll
+  for (int c = 0; c < C; ++c) v[c] = row[min(32 * c + lane, a.n_mels - 1)];
+  double xw[T];
+#pragma unroll
+  for (int t = 0; t < T; ++t) xw[t] = lane + 32 * t < NFFT ? (double)x[t] * w[t] : 0.0;
+#pragma unroll
+  for (int c = 0; c < C; ++c) {
+    if (32 * c >= a.n_mels) break;
+    const int mi = 32 * c + lane;
+    unsigned todo = __ballot_sync(FULL, mi < a.n_mels && v[c] * 1.4426950408889634f < thr);
+    while (todo) {
+      const int m = 32 * c + __ffs(todo) - 1;
+      todo &= todo - 1;
+      const int cnt = a.mel_cnt[m], lo = a.mel_lo[m], wo = a.mel_woff[m];
       double msum = 0.0;
 #pragma unroll 1
       for (int j = 0; j < cnt; ++j) {
-        const int k = a.mel_lo[m] + j;
-        double re = 0.0, im = 0.0;
-        int idx = (k * lane) % NFFT;   // (k n) mod 400 for n = lane + 32 t
-        const int step = (k * 32) % NFFT;
+        const int k = lo + j;
+        const double2 cs = a.fix_cs[(k * lane) % NFFT];   // (cos, sin) of 2 pi k n / 400 at n = lane
+        const double2 st = a.fix_cs[(k * 32) % NFFT];     // and of the 32-sample step
+        double cr = cs.x, sn = cs.y, re = 0.0, im = 0.0;
 #pragma unroll
         for (int t = 0; t < T; ++t) {
-          const double2 cs = a.fix_cs[idx];
-          re = fma(xw[t], cs.x, re);
-          im = fma(xw[t], cs.y, im);
-          idx += step;
-          if (idx >= NFFT) idx -= NFFT;
+          re = fma(xw[t], cr, re);
+          im = fma(xw[t], sn, im);
+          if (t + 1 < T) {
+            const double c2 = fma(cr, st.x, -sn * st.y);
+            sn = fma(sn, st.x, cr * st.y);
+            cr = c2;
+          }
         }
-#pragma unroll
+#pragma unroll 1
         for (int o = 16; o > 0; o >>= 1) {
           re += __shfl_xor_sync(FULL, re, o);
           im += __shfl_xor_sync(FULL, im, o);
         }
         // the weights carry the factor 1/4 of |2 X|^2
-        msum = fma(4.0 * (double)a.mel_w[a.mel_woff[m] + j], re * re + im * im, msum);
+        msum = fma(4.0 * (double)a.mel_w[wo + j], re * re + im * im, msum);
       }
-      __syncwarp();
-      if (lane == 0) orow[m] = msum < 1e-10 ? LOG_FLOOR : fmaxf(logf((float)msum), LOG_FLOOR);
-      __syncwarp();
+      if (lane == 0) row[m] = msum < 1e-10 ? LOG_FLOOR : fmaxf(logf((float)msum), LOG_FLOOR);
     }
   }
+  __syncwarp();
 }
 
 // ---------------------------------------------------------------------------
@@ -943,17 +967,15 @@ __device__ __forceinline__ void split_power(const Tables& tab, const cx& zk, con
   pm = fma2(qi, qi, mul2(qr, qr));
 }
 
-// Pass A for one thread (frames 2d and 2d + 1, role m2): windowed loads,
-// 20-point DFT over m1, twiddle; then, once the previous tile has released
-// the pass buffer (warp 0 waits for its row copies; group barrier), the
-// stores of the 20 outputs.  Returns the group's copy verdict (false: stop).
-// Offline tiles hold one utterance, so frame 2d + 1 starts one hop block
-// after frame 2d (slots of frames past the tile's end hold values whose
-// results are dropped); streaming tiles may pair frames of two streams, so
-// each frame's slots are looked up on their own.
+// Pass A for one thread (frames 2d and 2d + 1, role m2), in two steps.
+// pass_a_load: the windowed loads of the thread's 20 complex samples per
+// frame from the span.  Offline tiles hold one utterance, so frame 2d + 1
+// starts one hop block after frame 2d (slots of frames past the tile's end
+// hold values whose results are dropped); streaming tiles may pair frames of
+// two streams, so each frame's slots are looked up on their own.
 template <bool kOdd, bool kStream>
-__device__ __forceinline__ bool pass_a(const Tables& tab, const float* span, int eo, const Ctl& S, float4* Y,
-                                       int d, int m2, int warp, int grp) {
+__device__ __forceinline__ void pass_a_load(const Tables& tab, const float* span, int eo, const Ctl& S, int d, int m2,
+                                            cx (&z)[N1]) {
   const int off = 2 * m2 + (S.tma >> 2);
   const float* pa[3];
   const float* pb[3];
@@ -974,8 +996,20 @@ __device__ __forceinline__ bool pass_a(const Tables& tab, const float* span, int
     pb[1] = e + BLK;
     pb[2] = o + BLK;
   }
-  cx z[N1];
   window_load<kOdd>(z, pa, pb, tab, m2);
+}
+// Spans staged at an odd float offset: an out-of-line copy of the loads, so
+// that the common path keeps its register allocation.
+__device__ __noinline__ void pass_a_load_odd(const Tables& tab, const float* span, int eo, const Ctl& S, int d, int m2,
+                                             cx (&z)[N1]) {
+  pass_a_load<true, false>(tab, span, eo, S, d, m2, z);
+}
+// pass_a_store: the 20-point DFT over m1 and the twiddles; then, once the
+// previous tile has released the pass buffer (warp 0 waits for its row
+// copies; group barrier), the stores of the 20 outputs.  Returns the group's
+// copy verdict (false: stop).
+__device__ __forceinline__ bool pass_a_store(const Tables& tab, const Ctl& S, float4* Y, int d, int m2, int warp,
+                                             int grp, cx (&z)[N1]) {
   dft20(z);
 #pragma unroll
   for (int k1 = 1; k1 < N1; ++k1) {
@@ -1001,9 +1035,11 @@ __device__ __forceinline__ bool pass_a(const Tables& tab, const float* span, int
   }
   return true;
 }
-__device__ __noinline__ bool pass_a_odd(const Tables& tab, const float* span, int eo, const Ctl& S, float4* Y,
-                                        int d, int m2, int warp, int grp) {
-  return pass_a<true, false>(tab, span, eo, S, Y, d, m2, warp, grp);
+
+// A tile group's count of deferred frames, after the groups' regions
+// (recomputed where used rather than held in a register across the loop).
+__device__ __forceinline__ int* fixn_of(unsigned char* smem, const Args& a, int G, int grp) {
+  return reinterpret_cast<int*>(smem + TAB_BYTES + (size_t)G * a.group_bytes) + grp;
 }
 
 // kOddSpans: offline batches in which some utterance starts at an odd float
@@ -1032,11 +1068,15 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
   float* const Pbuf = reinterpret_cast<float*>(Y);   // power rows, after pass B has read Y
   float* const orows = Pbuf + PROWS_FLOATS;          // staged output rows, after the power rows
   float* const Sbuf = orows + TILE * orow_floats(a.n_mels);   // [MEL_WARPS][32]: frames' spectral energy
+  float* const Sthr = Sbuf + MEL_WARPS * TILE;                 // [32]: the guard's threshold per slot
+  unsigned* const Sflag = reinterpret_cast<unsigned*>(Sthr + TILE);   // the tile's flagged slots
+  const bool defer = !kStream && a.bulk_store && a.fixq_cap > 0;
   const int opitch = orow_floats(a.n_mels);
   int tile = blockIdx.x * G + grp;
   int armed0 = 0, armed1 = 0;   // COPY_TID: bulk-copy uses of each control buffer
 
   if (tid == COPY_TID) {
+    *fixn_of(smem_raw, a, G, grp) = 0;
     mbar_init(&ctl0->bar);
     mbar_init(&ctl1->bar);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -1069,11 +1109,11 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
     float4* dst = reinterpret_cast<float4*>(smem_raw);
     for (int i = threadIdx.x; i < (int)(sizeof(Tables) / 16); i += blockDim.x) dst[i] = src[i];
   }
-  if (!kStream && !a.meta_inline) {  // offline: this CTA's tile descriptors, searched in parallel
+  if constexpr (!kStream) {  // offline: this CTA's tile descriptors, searched in parallel
     const int rounds = (a.num_tiles + stride - 1) / stride;
     for (int j = threadIdx.x; j < rounds * G; j += blockDim.x) {
       const int t = blockIdx.x * G + (j % G) + (j / G) * stride;
-      if (t < a.num_tiles) a.tiles[t] = offline_desc(a, t);
+      if (t < a.num_tiles) a.tiles[t] = search_desc(a, t);
     }
   }
   __syncthreads();   // tables, descriptors and the initialised mbarriers
@@ -1081,7 +1121,7 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
   if (tile < a.num_tiles) {
     if (!ctl0->early) {
       if (tid == COPY_TID) {
-        if constexpr (!kStream) setup_offline(*ctl0, a, tile_desc(a, tile), span, kOddSpans);
+        if constexpr (!kStream) setup_offline(*ctl0, a, a.tiles[tile], span, kOddSpans);
         else setup_stream(*ctl0, a, tile);
         if (ctl0->tma) ctl0->bar_parity = (armed0++) & 1;
         ctl0->copy_ok = 1;
@@ -1089,15 +1129,14 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
       group_sync(grp);
       stage_tile<kStream>(*ctl0, span, tid, a);
     }
-    if (!kStream && tid == COPY_TID && tile + stride < a.num_tiles) ctl0->pending = tile_desc(a, tile + stride);
   }
   int cur = 0;
   for (; tile < a.num_tiles; tile += stride, cur ^= 1) {
     Ctl& S = cur ? *ctl1 : *ctl0;
     Ctl& N = cur ? *ctl0 : *ctl1;
     const int next = tile + stride;
-    TileDesc nd;   // the next tile's descriptor (used after pass A)
-    if (!kStream && tid == COPY_TID && next < a.num_tiles) nd = ctl0->pending;
+    TileDesc nd;   // the next tile's descriptor (loaded here, used after pass A)
+    if (!kStream && tid == COPY_TID && next < a.num_tiles) nd = a.tiles[next];
     // This tile's span: bulk copies complete on the mbarrier, which every
     // thread polls (bounded: ~65 ms) before it reads the span; a thread that
     // gives up clears the verdict, which the whole group reads after the
@@ -1114,17 +1153,15 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
 
 
     // ---- pass A: window, 20-point DFTs over m1, twiddle --------------------
-    // (spans staged at an odd float offset take a separate, out-of-line copy
-    // of the pass, so that the common path keeps its register allocation)
     {
-      const int sh = S.tma >> 2;   // the slots hold their samples from position sh
-      bool ok;
-      if constexpr (kOddSpans)
-        ok = (sh & 1) ? pass_a_odd(tab, span, a.eo_off, S, Y, d, role, warp, grp)
-                      : pass_a<false, kStream>(tab, span, a.eo_off, S, Y, d, role, warp, grp);
-      else
-        ok = pass_a<false, kStream>(tab, span, a.eo_off, S, Y, d, role, warp, grp);
-      if (!ok) {
+      cx z[N1];
+      if constexpr (kOddSpans) {
+        if ((S.tma >> 2) & 1) pass_a_load_odd(tab, span, a.eo_off, S, d, role, z);
+        else pass_a_load<false, kStream>(tab, span, a.eo_off, S, d, role, z);
+      } else {
+        pass_a_load<false, kStream>(tab, span, a.eo_off, S, d, role, z);
+      }
+      if (!pass_a_store(tab, S, Y, d, role, warp, grp, z)) {
         // a span copy did not complete in time: flag it, give copies still
         // in flight one more bounded wait (a slow copy must land before the
         // CTA's shared memory is released), and stop this group
@@ -1216,6 +1253,7 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
       q.x += __shfl_xor_sync(0xffffffffu, q.x, 8);
       q.y += __shfl_xor_sync(0xffffffffu, q.y, 8);
       if (((lane >> 3) & 1) == 0) *reinterpret_cast<float2*>(Sbuf + warp * TILE + 2 * d) = q;
+      if (tid == 0) *Sflag = 0u;
     }
     group_sync(grp);
 
@@ -1244,19 +1282,69 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
       for (int w = 0; w < MEL_WARPS; ++w) esum += Sbuf[w * TILE + lane];
       const float thr = lane < S.nslots ? lg2_approx(esum) + LG2_RISK_REL : __int_as_float(0xff800000);
       const bool risk = lo2 < thr;
-      if (__any_sync(0xffffffffu, risk))
-        mel_fixup(a, S, orows, opitch, a.warp_band[warp], a.warp_band[warp + 1], thr, risk, lane);
+      const unsigned rm = __ballot_sync(0xffffffffu, risk);
+      if (rm != 0u) {   // every warp finds the same threshold for a slot
+        if (risk) Sthr[lane] = thr;
+        if (lane == 0) atomicOr(Sflag, rm);
+      }
     }
-    if (a.bulk_store) fence_async_smem();   // the staged rows precede the bulk copies reading them
-    if (a.bulk_store && !kStream) {
-      // only warp 0, which issues the copies, waits for every warp's rows
-      if (warp == 0) group_wait2(grp);
-      else group_arrive2(grp);
+    if (defer) {
+      // the staged rows precede the bulk copies reading them; only warp 0,
+      // which issues the copies, waits for every warp's rows, and it queues
+      // the tile's flagged frames for after the group's last tile (or, with
+      // the queue full, recomputes them in place before the copies)
+      fence_async_smem();
+      if (warp == 0) {
+        group_wait2(grp);
+        const unsigned fm = *Sflag;
+        if (fm != 0u) {
+          const int n = *fixn_of(smem_raw, a, G, grp), k = __popc(fm);
+          if (n + k <= a.fixq_cap) {
+            if ((fm >> lane) & 1u) {
+              const Group& g = S.groups[0];
+              FixItem it;
+              it.src = (int64_t)(g.src0 - a.pcm) + (int64_t)HOP * lane;
+              it.row = (int)slot_row(S, lane);
+              it.thr = Sthr[lane];
+              a.fixq[(size_t)(blockIdx.x * G + grp) * a.fixq_cap + n + __popc(fm & ((1u << lane) - 1u))] = it;
+            }
+            __syncwarp();
+            if (lane == 0) *fixn_of(smem_raw, a, G, grp) = n + k;
+          } else {
+            for (unsigned r = fm; r != 0u; r &= r - 1u) {
+              const int f = __ffs(r) - 1;
+              fix_frame(a, S.groups[0].src0 + HOP * f, NFFT, nullptr, 0, orows + f * opitch, Sthr[f], lane);
+            }
+            fence_async_smem();
+          }
+        }
+      } else {
+        group_arrive2(grp);
+      }
     } else {
-      // every warp stores rows written by every warp; streaming: no thread
-      // overwrites a carry (below) while a warp's accuracy guard may still
-      // read the frames' samples from it
+      // every warp sees every warp's rows (the store below, the copies of
+      // warp 0), and the tile's flagged frames, which the warps recompute in
+      // place, one frame per warp in turn; streaming: no thread overwrites a
+      // carry (below) while a recomputation may still read the frames'
+      // samples from it
+      if (a.bulk_store) fence_async_smem();
       group_sync(grp);
+      const unsigned fm = *Sflag;
+      if (fm != 0u) {
+        int i = 0;
+        for (unsigned r = fm; r != 0u; r &= r - 1u, ++i) {
+          if (i % MEL_WARPS != warp) continue;
+          const int f = __ffs(r) - 1;
+          int gi = 0;   // the source holding frame slot f
+          for (int j = 0; j < S.ngroups; ++j)
+            if (f >= S.groups[j].slot0 && f < S.groups[j].slot0 + S.groups[j].nframes) gi = j;
+          const Group& g = S.groups[gi];
+          fix_frame(a, g.src0, g.len0, g.src1, g.start + (int64_t)HOP * (f - g.slot0), orows + f * opitch, Sthr[f],
+                    lane);
+        }
+        if (a.bulk_store) fence_async_smem();
+        group_sync(grp);
+      }
     }
 
     // ---- store: the staged rows of the tile's frames ---------------------
@@ -1282,9 +1370,6 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
         }
       }
     }
-    // the descriptor of this group's tile after next, found while warp 0
-    // issues the row copies (used after the next tile's pass A)
-    if (!kStream && tid == COPY_TID && next + stride < a.num_tiles) ctl0->pending = tile_desc(a, next + stride);
     if constexpr (kStream) {
       // each owned stream's new carry, from the span (the mel stage's
       // accuracy guard may have read the frames' samples from the old
@@ -1307,6 +1392,21 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
     }
   }
   if (warp == 0) asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");   // rows written before exit
+  if (defer) {
+    // the group's deferred frames, one per warp in turn, recomputed in the
+    // output rows once the row copies have landed (warp 0, which queued the
+    // frames and issued the copies, orders the copies' writes before the
+    // recomputation's reads and writes only when there is a frame: the
+    // proxy fence costs about 2 us)
+    if (warp == 0 && *fixn_of(smem_raw, a, G, grp) > 0) asm volatile("fence.proxy.async.global;\n" ::: "memory");
+    group_sync(grp);
+    const int n = *fixn_of(smem_raw, a, G, grp);
+    const FixItem* q = a.fixq + (size_t)(blockIdx.x * G + grp) * a.fixq_cap;
+    for (int i = warp; i < n; i += MEL_WARPS) {
+      const FixItem it = q[i];
+      fix_frame(a, a.pcm + it.src, NFFT, nullptr, 0, a.out + (int64_t)it.row * a.n_mels, it.thr, lane);
+    }
+  }
 }
 
 }  // namespace logmel
