@@ -631,18 +631,31 @@ __device__ void setup_offline(Ctl& S, const Args& a, const TileDesc& t, const fl
 __device__ void setup_stream(Ctl& S, const Args& a, int tile) {
   int ng = 0, slot = 0, block = 0;
   const int sg = tile / a.tps, st = tile - sg * a.tps;
-  for (int j = 0; j < a.spt; ++j) {
+  // the tile's streams' carry lengths and chunk bounds, all loaded before
+  // the first is used (one memory latency, not one per stream)
+  constexpr int SPT_MAX = 4;
+  int cl[SPT_MAX];
+  int64_t o0[SPT_MAX], o1[SPT_MAX];
+#pragma unroll
+  for (int j = 0; j < SPT_MAX; ++j) {
+    const int sl = min(sg * a.spt + j, a.n_push_streams - 1);
+    cl[j] = a.carry_len[a.stream_base + sl];
+    o0[j] = a.push_off != nullptr ? a.push_off[sl] : 0;
+    o1[j] = a.push_off != nullptr ? a.push_off[sl + 1] : 0;
+  }
+#pragma unroll
+  for (int j = 0; j < SPT_MAX; ++j) {
     const int sl = sg * a.spt + j;
-    if (sl >= a.n_push_streams) break;
+    if (j >= a.spt || sl >= a.n_push_streams) break;
     const int s = a.stream_base + sl;
     int64_t len = a.push_len;
     const float* chunk = a.chunks + (int64_t)sl * a.chunk_stride;
     if (a.push_off != nullptr) {
-      chunk = a.chunks + a.push_off[sl];
-      len = a.push_off[sl + 1] - a.push_off[sl];
+      chunk = a.chunks + o0[j];
+      len = o1[j] - o0[j];
       if (len == 0) continue;   // nothing arrives: the stream's state stays as it is
     }
-    const int c = a.carry_len[s];
+    const int c = cl[j];
     const int64_t B = c + len;
     const int64_t n = B >= NFFT ? (B - NFFT) / HOP + 1 : 0;
     const int64_t f0 = (int64_t)st * TILE;
@@ -998,12 +1011,6 @@ __device__ __forceinline__ void pass_a_load(const Tables& tab, const float* span
   }
   window_load<kOdd>(z, pa, pb, tab, m2);
 }
-// Spans staged at an odd float offset: an out-of-line copy of the loads, so
-// that the common path keeps its register allocation.
-__device__ __noinline__ void pass_a_load_odd(const Tables& tab, const float* span, int eo, const Ctl& S, int d, int m2,
-                                             cx (&z)[N1]) {
-  pass_a_load<true, false>(tab, span, eo, S, d, m2, z);
-}
 // pass_a_store: the 20-point DFT over m1 and the twiddles; then, once the
 // previous tile has released the pass buffer (warp 0 waits for its row
 // copies; group barrier), the stores of the 20 outputs.  Returns the group's
@@ -1034,6 +1041,21 @@ __device__ __forceinline__ bool pass_a_store(const Tables& tab, const Ctl& S, fl
     yrow[k1 * YROW] = make_float4(v.re.x, v.re.y, v.im.x, v.im.y);
   }
   return true;
+}
+
+// The whole pass A for one thread; spans staged at an odd float offset take
+// an out-of-line copy of it (its 20 complex values stay in that copy's
+// registers), so that the common path keeps its register allocation.
+template <bool kOdd, bool kStream>
+__device__ __forceinline__ bool pass_a(const Tables& tab, const float* span, int eo, const Ctl& S, float4* Y, int d,
+                                       int m2, int warp, int grp) {
+  cx z[N1];
+  pass_a_load<kOdd, kStream>(tab, span, eo, S, d, m2, z);
+  return pass_a_store(tab, S, Y, d, m2, warp, grp, z);
+}
+__device__ __noinline__ bool pass_a_odd(const Tables& tab, const float* span, int eo, const Ctl& S, float4* Y,
+                                        int d, int m2, int warp, int grp) {
+  return pass_a<true, false>(tab, span, eo, S, Y, d, m2, warp, grp);
 }
 
 // A tile group's count of deferred frames, after the groups' regions
@@ -1154,14 +1176,13 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
 
     // ---- pass A: window, 20-point DFTs over m1, twiddle --------------------
     {
-      cx z[N1];
-      if constexpr (kOddSpans) {
-        if ((S.tma >> 2) & 1) pass_a_load_odd(tab, span, a.eo_off, S, d, role, z);
-        else pass_a_load<false, kStream>(tab, span, a.eo_off, S, d, role, z);
-      } else {
-        pass_a_load<false, kStream>(tab, span, a.eo_off, S, d, role, z);
-      }
-      if (!pass_a_store(tab, S, Y, d, role, warp, grp, z)) {
+      bool ok;
+      if constexpr (kOddSpans)
+        ok = ((S.tma >> 2) & 1) ? pass_a_odd(tab, span, a.eo_off, S, Y, d, role, warp, grp)
+                                : pass_a<false, kStream>(tab, span, a.eo_off, S, Y, d, role, warp, grp);
+      else
+        ok = pass_a<false, kStream>(tab, span, a.eo_off, S, Y, d, role, warp, grp);
+      if (!ok) {
         // a span copy did not complete in time: flag it, give copies still
         // in flight one more bounded wait (a slow copy must land before the
         // CTA's shared memory is released), and stop this group
