@@ -460,7 +460,9 @@ static cudaError_t launch(const logmel_plan* p, Args& a, int64_t tiles, cudaStre
   std::memcpy(a.mel_cnt, p->mel.mel_cnt, sizeof a.mel_cnt);
   std::memcpy(a.mel_woff, p->mel.mel_woff, sizeof a.mel_woff);
   std::memcpy(a.warp_band, p->mel.warp_band, sizeof a.warp_band);
-  const int grid = (int)std::min<int64_t>((tiles + c.groups - 1) / c.groups, c.max_ctas);
+  // one CTA per tile up to the resident limit: a batch of fewer tiles than
+  // the device has SMs runs one tile group per SM (the others idle)
+  const int grid = (int)std::min<int64_t>(tiles, c.max_ctas);
   const int block = c.groups * GROUP_THREADS;
   // offline: each tile group queues its flagged frames (when the queue
   // covers every group of the grid)

@@ -1094,7 +1094,10 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
   unsigned* const Sflag = reinterpret_cast<unsigned*>(Sthr + TILE);   // the tile's flagged slots
   const bool defer = !kStream && a.bulk_store && a.fixq_cap > 0;
   const int opitch = orow_floats(a.n_mels);
-  int tile = blockIdx.x * G + grp;
+  // tile groups are numbered group-major across the grid (all CTAs' group
+  // 0, then their group 1, ...), so a last, partial round of tiles spreads
+  // over the SMs one group each before any SM runs two of them
+  int tile = grp * (int)gridDim.x + blockIdx.x;
   int armed0 = 0, armed1 = 0;   // COPY_TID: bulk-copy uses of each control buffer
 
   if (tid == COPY_TID) {
@@ -1134,7 +1137,7 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
   if constexpr (!kStream) {  // offline: this CTA's tile descriptors, searched in parallel
     const int rounds = (a.num_tiles + stride - 1) / stride;
     for (int j = threadIdx.x; j < rounds * G; j += blockDim.x) {
-      const int t = blockIdx.x * G + (j % G) + (j / G) * stride;
+      const int t = (j % G) * (int)gridDim.x + blockIdx.x + (j / G) * stride;
       if (t < a.num_tiles) a.tiles[t] = search_desc(a, t);
     }
   }
