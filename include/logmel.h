@@ -245,7 +245,9 @@ logmel_status logmel_stream_reset(logmel_stream* st, int stream_id, void* stream
  * reached the copy (a copy from pageable memory returns once its source has
  * been consumed), and the next call rewrites the buffer.  Batches of up to
  * 256 utterances carry their metadata in the kernel launch and do not block.
- * No device or pinned memory is allocated or freed. */
+ * Only those calls may be captured into a CUDA graph: a captured call of
+ * more than 256 utterances would replay a copy of whatever the host buffer
+ * holds at replay time.  No device or pinned memory is allocated or freed. */
 logmel_status logmel_compute_noalloc(const float* pcm, const int64_t* offsets, int64_t n_utt,
                                      float* out, int* device_status, void* stream);
 
