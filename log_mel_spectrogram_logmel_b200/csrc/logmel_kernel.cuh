@@ -131,6 +131,7 @@ struct __align__(16) FixItem {
 };
 constexpr int FIXQ_CAP = 16;   // deferred frames per tile group
 constexpr int FIXN_BYTES = 16;  // shared memory after the groups' regions: each group's count of deferred frames
+constexpr int FIXN_FULL = 1 << 30;   // set in a group's count once its queue has overflowed
 
 struct Args {
   // offline: tensor views of the PCM for the tile copies, one per parity q
@@ -1312,11 +1313,15 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
         if (lane == 0) atomicOr(Sflag, rm);
       }
     }
-    if (defer) {
+    // (every warp reads the group's count after the same barriers, before
+    // warp 0 may change it below: the choice is uniform)
+    if (defer && !(*fixn_of(smem_raw, a, G, grp) & FIXN_FULL)) {
       // the staged rows precede the bulk copies reading them; only warp 0,
       // which issues the copies, waits for every warp's rows, and it queues
-      // the tile's flagged frames for after the group's last tile (or, with
-      // the queue full, recomputes them in place before the copies)
+      // the tile's flagged frames for after the group's last tile (or, when
+      // they overflow the queue, recomputes them in place before the copies
+      // and marks the queue full: the group's later tiles take the branch
+      // below, where every warp recomputes)
       fence_async_smem();
       if (warp == 0) {
         group_wait2(grp);
@@ -1340,6 +1345,7 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
               fix_frame(a, S.groups[0].src0 + HOP * f, NFFT, nullptr, 0, orows + f * opitch, Sthr[f], lane);
             }
             fence_async_smem();
+            if (lane == 0) *fixn_of(smem_raw, a, G, grp) = n | FIXN_FULL;
           }
         }
       } else {
@@ -1422,9 +1428,10 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
     // frames and issued the copies, orders the copies' writes before the
     // recomputation's reads and writes only when there is a frame: the
     // proxy fence costs about 2 us)
-    if (warp == 0 && *fixn_of(smem_raw, a, G, grp) > 0) asm volatile("fence.proxy.async.global;\n" ::: "memory");
+    if (warp == 0 && (*fixn_of(smem_raw, a, G, grp) & ~FIXN_FULL) > 0)
+      asm volatile("fence.proxy.async.global;\n" ::: "memory");
     group_sync(grp);
-    const int n = *fixn_of(smem_raw, a, G, grp);
+    const int n = *fixn_of(smem_raw, a, G, grp) & ~FIXN_FULL;
     const FixItem* q = a.fixq + (size_t)(blockIdx.x * G + grp) * a.fixq_cap;
     for (int i = warp; i < n; i += MEL_WARPS) {
       const FixItem it = q[i];

@@ -288,3 +288,14 @@ def test_accuracy_guard_on_pure_tones(lib, plan):
     g80 = _run(p80, x, [0, len(x)])
     L80, M80 = O.log_mel(x, O.Params(n_mels=80, fmin=20.0, fmax=7600.0), return_energy=True)
     check_against_oracle(g80, L80, M80)
+
+
+def test_accuracy_guard_after_the_queue_overflows(plan):
+    """160 s of the same tones: 500 tiles, so some tile groups run two. A
+    group's first tile overflows its queue of deferred frames; from then on
+    every warp of the group recomputes its tiles' flagged frames in place."""
+    x = W.page1_test_tones(160.0)
+    g = _run(plan, x, [0, len(x)])
+    L, M = O.log_mel(x, return_energy=True)
+    assert g.shape[0] == 15998
+    check_against_oracle(g, L, M)
