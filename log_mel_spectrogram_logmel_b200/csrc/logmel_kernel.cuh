@@ -428,6 +428,9 @@ static_assert(TAB_BYTES + MAX_TILE_GROUPS * group_bytes_for(OFFLINE_SPAN_BLOCKS,
 // so their 8-byte pair stores hit distinct banks).
 __device__ __forceinline__ int pcol(int f, int par) { return f ^ (16 * par); }
 
+// bar.sync / bar.arrive are the warp-aligned forms: every lane of a warp must
+// execute the same one.  Where a barrier follows a block that one lane (the
+// copy thread) runs alone, the warp reconverges first (__syncwarp).
 __device__ __forceinline__ void group_sync(int g) {
   asm volatile("bar.sync %0, %1;" ::"r"(g + 1), "r"(GROUP_THREADS) : "memory");
 }
@@ -1127,6 +1130,7 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
   if constexpr (kStream) {
     // a push is one or two tiles per group: its first span copy (cp.async
     // by the whole group) leaves before the tables are staged
+    __syncwarp();
     group_sync(grp);
     if (tile < a.num_tiles) stage_tile<kStream>(*ctl0, span, tid, a);
   }
@@ -1152,6 +1156,7 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
         if (ctl0->tma) ctl0->bar_parity = (armed0++) & 1;
         ctl0->copy_ok = 1;
       }
+      __syncwarp();
       group_sync(grp);
       stage_tile<kStream>(*ctl0, span, tid, a);
     }
@@ -1203,6 +1208,7 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
       if (N.tma) N.bar_parity = cur ? (armed0++) & 1 : (armed1++) & 1;
       N.copy_ok = 1;
     }
+    __syncwarp();
     group_sync(grp);
 
     // every thread has finished reading the span (its values were consumed
@@ -1416,6 +1422,7 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
         if (tid == 0) *g.carry_len_dst = g.new_carry_len;
       }
       if (next < a.num_tiles) {
+        __syncwarp();
         group_sync(grp);   // the span has been read
         stage_tile<kStream>(N, span, tid, a);
       }
