@@ -452,6 +452,11 @@ __device__ __forceinline__ void cp_async8(float* dst, const float* src) {
   const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(dst));
   asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(d), "l"(src) : "memory");
 }
+// 16 bytes, L2 only (both addresses 16-byte aligned).
+__device__ __forceinline__ void cp_async16(float* dst, const float* src) {
+  const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(src) : "memory");
+}
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
 }
@@ -771,7 +776,22 @@ __device__ __forceinline__ void stage_tile(Ctl& S, float* span, int tid, const A
         if (tid + HOP * q < n) cp_async4(blk_addr(span, eo, g.block0 + q) + tid, base + tid + HOP * q);
     } else {
       // streaming (carry ++ chunk): a push stages far fewer samples than the
-      // span holds, so the loop runs over the staged hop blocks only
+      // span holds, so the loops run over the staged samples only.  With the
+      // carry length, the staged length and both sources on the 4-sample
+      // grid (an 80 ms clock keeps a 240-sample carry), 16-byte copies, no
+      // copy straddling carry and chunk; else 4-byte ones
+      if constexpr (kStream) {
+        if (((g.len0 | n) & 3) == 0 &&
+            ((reinterpret_cast<uintptr_t>(g.src0) | reinterpret_cast<uintptr_t>(g.src1)) & 15) == 0) {
+          for (int i = tid; 4 * i < n; i += THREADS) {
+            const int p = 4 * i, q = p / HOP;
+            const int64_t pos = g.start + p;
+            cp_async16(blk_addr(span, eo, g.block0 + q) + (p - q * HOP),
+                       pos < g.len0 ? g.src0 + pos : g.src1 + (pos - g.len0));
+          }
+          continue;
+        }
+      }
 #pragma unroll 2
       for (int q = 0; HOP * q < n; ++q) {
         const int64_t pos = g.start + tid + HOP * q;
