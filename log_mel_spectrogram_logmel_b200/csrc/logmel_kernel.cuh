@@ -1123,6 +1123,12 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
   // over the SMs one group each before any SM runs two of them
   int tile = grp * (int)gridDim.x + blockIdx.x;
   int armed0 = 0, armed1 = 0;   // COPY_TID: bulk-copy uses of each control buffer
+  {  // FFT tables -> shared memory, once per CTA, asynchronously (waited before the prologue's barrier)
+    const float* src = reinterpret_cast<const float*>(a.tables);
+    float* dst = reinterpret_cast<float*>(smem_raw);
+    for (int i = threadIdx.x; i < (int)(sizeof(Tables) / 16); i += blockDim.x) cp_async16(dst + 4 * i, src + 4 * i);
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+  }
 
   if (tid == COPY_TID) {
     *fixn_of(smem_raw, a, G, grp) = 0;
@@ -1154,11 +1160,6 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
     group_sync(grp);
     if (tile < a.num_tiles) stage_tile<kStream>(*ctl0, span, tid, a);
   }
-  {  // FFT tables -> shared memory, once per CTA
-    const float4* src = reinterpret_cast<const float4*>(a.tables);
-    float4* dst = reinterpret_cast<float4*>(smem_raw);
-    for (int i = threadIdx.x; i < (int)(sizeof(Tables) / 16); i += blockDim.x) dst[i] = src[i];
-  }
   if constexpr (!kStream) {  // offline: this CTA's tile descriptors, searched in parallel
     const int rounds = (a.num_tiles + stride - 1) / stride;
     for (int j = threadIdx.x; j < rounds * G; j += blockDim.x) {
@@ -1166,6 +1167,7 @@ __global__ void __launch_bounds__(GROUP_THREADS * MAX_TILE_GROUPS, 1) logmel_fus
       if (t < a.num_tiles) a.tiles[t] = search_desc(a, t);
     }
   }
+  asm volatile("cp.async.wait_all;\n" ::: "memory");   // this thread's table (and cp.async span) copies
   __syncthreads();   // tables, descriptors and the initialised mbarriers
 
   if (tile < a.num_tiles) {
