@@ -111,9 +111,13 @@ logmel_status logmel_frame_offsets(const logmel_plan* plan, const int64_t* offse
  * launches one kernel.  For n_utt <= 256 the per-utterance offsets travel in
  * the launch parameters; larger batches first copy them host->device on
  * `stream` (from a pinned ring owned by the plan).  It does not synchronise
- * unless the plan's scratch must grow (first call with a larger batch of
- * more than 256 utterances), which synchronises the device.  n_utt == 0 or
- * total_frames == 0 is a no-op. */
+ * unless the plan's scratch must grow (the first call with more 32-frame
+ * tiles, or more than 256 utterances, than any call before it), which
+ * synchronises the device.  The kernel writes the plan's device scratch (tile
+ * descriptors, and the queue of frames whose bands it recomputes in float64),
+ * so calls on one plan whose work could overlap on the GPU (two streams) must
+ * be ordered, for example on one stream.  n_utt == 0 or total_frames == 0 is
+ * a no-op. */
 logmel_status logmel_compute(logmel_plan* plan, const float* pcm, const int64_t* offsets,
                              int64_t n_utt, float* out, void* stream);
 
