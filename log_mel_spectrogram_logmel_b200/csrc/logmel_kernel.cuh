@@ -34,6 +34,11 @@
 //           in a fixed order (fully unrolled for the default 128-band
 //           filterbank, weights as immediates)
 //   log     ln = lg2 * ln 2, clamped below at the fp32 value of ln(1e-10)
+//   guard   pass B also sums each frame's spectral energy S; a band whose
+//           energy lies under 3.75e-10 S (out of fp32's reach) is
+//           recomputed in float64 from the frame's samples (fix_frame):
+//           offline after the tile group's last tile, from a queue, and
+//           streaming inside its tile
 //   store   each frame's row of n_mels fp32 is staged in shared memory by
 //           16-byte stores (four bands) and leaves through one 2-D tensor
 //           copy per full tile, else one bulk copy per row
@@ -778,7 +783,7 @@ __device__ __forceinline__ void stage_tile(Ctl& S, float* span, int tid, const A
       // streaming (carry ++ chunk): a push stages far fewer samples than the
       // span holds, so the loops run over the staged samples only.  With the
       // carry length, the staged length and both sources on the 4-sample
-      // grid (an 80 ms clock keeps a 240-sample carry), 16-byte copies, no
+      // grid (an 80 ms clock keeps every carry at 320 samples), 16-byte copies, no
       // copy straddling carry and chunk; else 4-byte ones
       if constexpr (kStream) {
         if (((g.len0 | n) & 3) == 0 &&
